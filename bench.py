@@ -1,0 +1,358 @@
+#!/usr/bin/env python
+"""Throughput of the gated MLA hot path on B200.
+
+One step = one causal gated attention forward with the fused per-head max
+logit on the long-context workload (B=1, T=16384, H=96, d_qk=192, d_v=128,
+bf16, heads 0-7 x4), plus one absorbed-latent decode of 64 sequences with
+context lengths U[1024, 8192] over the 576-wide latent cache.  ``value`` is
+the forward's TFLOP/s (causal half including the diagonal: 2*B*H*T(T+1)/2*320
+FLOP per call); the decode's HBM GB/s is reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own independent problem instance
+(weak scaling: the path partitions by independent problems); the per-head max
+logits are MAX-all-reduced each step, the one exchange data parallelism adds.
+``--impl reference`` times the CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal MLA fwd TFLOP/s (+maxlogit) at T=16k; absorbed decode HBM GB/s"
+B_FWD, T_FWD = 1, 16384
+FWD_FLOP = 2.0 * B_FWD * 96 * T_FWD * (T_FWD + 1) / 2 * (192 + 128)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d.get("bf16_tflops_sustained"),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+def host_cores():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count()
+    threads = n
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            threads = max(i.get("num_threads", n) for i in info)
+    except Exception:
+        pass
+    return threads
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(inp, rows_per_step=96):
+    """Oracle attention for the heaviest query rows of head 0 (a bounded sample).
+
+    Returns (seconds, flop) where flop counts the causal work of those rows."""
+    import numpy as np
+    import oracle
+    T = inp["Q"].shape[1]
+    rows = [(0, t, 0) for t in range(T - rows_per_step, T)]
+    flop = sum(2.0 * (t + 1) * 320 for (_, t, _) in rows)
+    t0 = time.perf_counter()
+    oracle.attention_rows(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"], rows)
+    return time.perf_counter() - t0, flop
+
+
+def cpu_baseline(inp, target_s=12.0):
+    secs, flops = 0.0, 0.0
+    n = 0
+    while secs < target_s:
+        s, f = oracle_sample(inp)
+        secs += s
+        flops += f
+        n += 1
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"{n} x 96 causal rows (t = 16288..16383) of head 0 at B=1,T=16384, float64 numpy; "
+                      f"{secs:.1f} s of CPU work"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from gated_mla_qk_b200 import synth
+    inp = synth.attn_core(B_FWD, T_FWD, synth.K3, seed=2, hot_heads=8, hot_scale=4.0)
+    for _ in range(args.warmup):
+        oracle_sample(inp, rows_per_step=32)
+    tot_s, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        s, f = oracle_sample(inp, rows_per_step=32)
+        tot_s += s
+        tot_f += f
+    v = tot_f / tot_s / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "attention core B=1 T=16384 H=96 (bounded sample per step: 32 heaviest rows of head 0)",
+                       "B": B_FWD, "T": T_FWD, "H": 96},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+                             "sample": "per step: causal rows t=16352..16383 of head 0, float64 numpy"},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import numpy as np
+    import torch
+    import gated_mla_qk_b200 as gm
+    from gated_mla_qk_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    gm.load_library()
+
+    # ---- inputs (seeded; each rank its own independent problem) ----
+    geom = synth.K3
+    inp = synth.attn_core(B_FWD, T_FWD, geom, seed=2 + 1000 * rank, hot_heads=8, hot_scale=4.0)
+    dq = {k: synth.to_torch(v, "bf16", "cuda") for k, v in inp.items()}
+    O = torch.empty(B_FWD, T_FWD, geom.H * geom.d_v, dtype=torch.bfloat16, device="cuda")
+    ml = torch.empty(geom.H, dtype=torch.float32, device="cuda")
+    dec = synth.decode_batch(seed=4 + 1000 * rank)
+    dd = dict(q=synth.to_torch(dec["q"], "bf16", "cuda"), W_UKV=synth.to_torch(dec["W_UKV"], "bf16", "cuda"),
+              cache=synth.to_torch(dec["cache"], "bf16", "cuda"), offs=torch.from_numpy(dec["seq_offsets"]).cuda())
+    max_len = int(dec["lens"].max())
+    Od = torch.empty(64, geom.H, geom.d_v, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(gm.mla_decode_workspace(geom, gm.GMLA_BF16, 64, max_len), dtype=torch.uint8, device="cuda")
+    total_tokens = int(dec["seq_offsets"][-1])
+    dec_bytes_cache = total_tokens * 576 * 2
+    dec_bytes = dec_bytes_cache + 2 * 512 * 96 * 128 * 2 + 64 * 96 * (192 + 128) * 2
+    st = torch.cuda.current_stream()
+
+    def fwd():
+        gm.mla_attn_fwd(geom, dq["Q"], dq["KC"], dq["kS"], dq["V"], dq["g"], O, ml)
+
+    def decode():
+        gm.mla_decode_absorbed(geom, dd["q"], dd["W_UKV"], dd["cache"], dd["offs"], max_len, None, Od, ws)
+
+    def step(ev):
+        ev[0].record(st)
+        fwd()
+        ev[1].record(st)
+        if dist is not None:
+            dist.all_reduce(ml, op=dist.ReduceOp.MAX)
+        ev[2].record(st)
+        decode()
+        ev[3].record(st)
+
+    for _ in range(args.warmup):
+        fwd(); decode()
+    torch.cuda.synchronize()
+    assert gm.device_status() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = gm.launch_count()
+    with ClockSampler(local) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(st)
+        for k in range(args.steps):
+            step(evs[k])
+        end.record(st)
+        torch.cuda.synchronize()
+    launches = gm.launch_count() - n0
+    if dist is not None:
+        dist.barrier()
+    status = gm.device_status()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    t = torch.tensor([total_ms, sum(fwd_ms), sum(dec_ms)], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_sum, dec_sum = t.tolist()
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: dq[k].cpu().pin_memory() for k in ("Q", "KC", "kS", "V", "g")}
+        O_h = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        ml_h = torch.empty(ml.shape, dtype=ml.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pin.values())
+        d2h = O_h.numel() * O_h.element_size() + ml_h.numel() * 4
+        dev_in = {k: torch.empty_like(dq[k]) for k in pin}
+        del dq
+        e_steps = max(2, min(args.steps, 5))
+        for _ in range(1):
+            for k in pin:
+                dev_in[k].copy_(pin[k], non_blocking=True)
+            gm.mla_attn_fwd(geom, dev_in["Q"], dev_in["KC"], dev_in["kS"], dev_in["V"], dev_in["g"], O, ml)
+            O_h.copy_(O, non_blocking=True); ml_h.copy_(ml, non_blocking=True)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(e_steps):
+            for k in pin:
+                dev_in[k].copy_(pin[k], non_blocking=True)
+            gm.mla_attn_fwd(geom, dev_in["Q"], dev_in["KC"], dev_in["kS"], dev_in["V"], dev_in["g"], O, ml)
+            O_h.copy_(O, non_blocking=True); ml_h.copy_(ml, non_blocking=True)
+        b.record(st)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([a.elapsed_time(b) / e_steps], dtype=torch.float64, device="cuda")
+        if dist is not None:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * FWD_FLOP / (e_ms.item() / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms.item(),
+               "what": "mla_attn_fwd with inputs copied from pinned host memory and O + maxlogit copied back"}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    pk = peaks()
+    fwd_avg_ms = fwd_sum / args.steps
+    dec_avg_ms = dec_sum / args.steps
+    fwd_tflops = FWD_FLOP / (fwd_avg_ms / 1e3) / 1e12
+    dec_gbs = dec_bytes / (dec_avg_ms / 1e3) / 1e9
+    prof_traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        prof_traffic = json.load(open(tp)).get("attn_fwd_T16384")
+    line = {
+        "metric": METRIC,
+        "value": world * fwd_tflops,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "gated MLA attention fwd + maxlogit, B=1 T=16384 H=96 d_qk=192 d_v=128 bf16 "
+                               "(heads 0-7 x4); plus absorbed decode 64 seqs L~U[1024,8192] H=96",
+                   "B": B_FWD, "T": T_FWD, "H": 96, "decode_tokens": total_tokens,
+                   "l2": "inputs larger than L2 (fwd inputs 1.8 GB, decode cache %.0f MB); no flush" % (dec_bytes_cache / 1e6),
+                   "parallelism": f"replicas x{world} (independent problems), maxlogit MAX all-reduce"},
+        "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
+                     "frac": fwd_tflops / pk["bf16"], "traffic": prof_traffic,
+                     "kernel": "tc_attn::attn_fwd_kernel", "peak_source": f"{pk['src']} bf16 burst",
+                     "frac_of_sustained": fwd_tflops / pk["bf16_sust"] if pk["bf16_sust"] else None},
+        "decode": {"value": world * dec_gbs, "unit": "GB/s", "ms": dec_avg_ms,
+                   "bytes_per_call": dec_bytes, "cache_only_gbs": dec_bytes_cache / (dec_avg_ms / 1e3) / 1e9,
+                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                "frac": dec_gbs / pk["hbm"]}},
+        "fwd_ms": fwd_avg_ms,
+        "gpu_launches": launches,
+        "device_status": status,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

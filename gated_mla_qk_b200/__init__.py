@@ -1,0 +1,209 @@
+"""Python binding of libgmla.so (the C ABI in include/gmla.h).
+
+Argument marshalling only: every function takes torch tensors that already
+live on the GPU, checks dtype / contiguity, and passes raw device pointers and
+the current CUDA stream to the library, which runs every step of the path in
+its own kernels.  There is no CPU or library fallback: if the shared object is
+missing, importing the binding's functions raises.
+
+Entry points (same names as the C ABI): ``mla_up_proj``, ``mla_attn_fwd``,
+``qkclip_rescale``, ``mla_decode_absorbed``, ``mla_gemm``; plus the workspace
+size queries, ``device_status`` and ``launch_count``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .synth import Geom, K3, TINY  # noqa: F401  (geometry type shared with callers)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgmla.so")
+
+GMLA_BF16, GMLA_F32 = 0, 1
+STATUS = {0: "GMLA_OK", -1: "GMLA_EINVAL", -2: "GMLA_EALIGN", -3: "GMLA_EUNSUPPORTED", -4: "GMLA_ECUDA",
+          -5: "GMLA_ETIMEOUT", -6: "GMLA_EWORKSPACE"}
+
+EXPORTS = ["mla_up_proj_workspace", "mla_up_proj", "mla_attn_fwd", "qkclip_rescale", "mla_decode_workspace",
+           "mla_decode_absorbed", "mla_gemm", "gmla_device_status", "gmla_last_cuda_error", "gmla_strerror",
+           "gmla_version", "gmla_launch_count"]
+
+
+class GmlaError(RuntimeError):
+    def __init__(self, fn: str, status: int, lib=None):
+        msg = f"{fn} failed: {STATUS.get(status, status)}"
+        if lib is not None:
+            msg += f" ({lib.gmla_strerror(status).decode()})"
+            if status == -4:
+                msg += f", cudaError {lib.gmla_last_cuda_error()}"
+        super().__init__(msg)
+        self.status = status
+
+
+class CGeom(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int), ("d_model", ctypes.c_int), ("q_lora", ctypes.c_int), ("kv_lora", ctypes.c_int),
+                ("d_c", ctypes.c_int), ("d_s", ctypes.c_int), ("d_v", ctypes.c_int), ("rms_eps", ctypes.c_float)]
+
+    @classmethod
+    def of(cls, g: Geom) -> "CGeom":
+        return cls(g.H, g.d_model, g.q_lora, g.kv_lora, g.d_c, g.d_s, g.d_v, g.rms_eps)
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libgmla.so and declare its signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m gated_mla_qk_b200.build` "
+                          "(there is no fallback implementation)")
+    lib = ctypes.CDLL(path)
+    P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    G = ctypes.POINTER(CGeom)
+    sig = {
+        "mla_up_proj_workspace": (S, [G, I, I, I]),
+        "mla_up_proj": (I, [G, I, I, I] + [P] * 12 + [P, S, P]),
+        "mla_attn_fwd": (I, [G, I, I, I, P, P, P, P, P, P, P, P]),
+        "qkclip_rescale": (I, [G, I, P, P, P, F, P, P, P]),
+        "mla_decode_workspace": (S, [G, I, I, I]),
+        "mla_decode_absorbed": (I, [G, I, I, P, P, P, P, I, P, P, P, S, P]),
+        "mla_gemm": (I, [I, I, I, I, P, P, P, P]),
+        "gmla_device_status": (I, [P]),
+        "gmla_last_cuda_error": (I, []),
+        "gmla_strerror": (ctypes.c_char_p, [I]),
+        "gmla_version": (I, []),
+        "gmla_launch_count": (ctypes.c_ulonglong, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return GMLA_BF16
+    if t.dtype == torch.float32:
+        return GMLA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t, name, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(fn, status):
+    if status != 0:
+        raise GmlaError(fn, status, _lib)
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+def mla_up_proj_workspace(geom: Geom, dtype_code: int, B: int, T: int) -> int:
+    return load_library().mla_up_proj_workspace(ctypes.byref(CGeom.of(geom)), dtype_code, B, T)
+
+
+def mla_up_proj(geom: Geom, x, W_DQ, w_q, W_UQ, W_DKV, w_kv, W_UKV, Q, KC, kS, V, cache=None, workspace=None,
+                stream=None):
+    """Fill Q, KC, kS, V (and the latent cache if given) from x; see include/gmla.h."""
+    lib = load_library()
+    B, T = x.shape[0], x.shape[1]
+    dt = _dtype_code(x)
+    need = mla_up_proj_workspace(geom, dt, B, T)
+    if workspace is None:
+        workspace = _torch().empty(need, dtype=_torch().uint8, device=x.device)
+    _check("mla_up_proj", lib.mla_up_proj(
+        ctypes.byref(CGeom.of(geom)), dt, B, T,
+        *[_ptr(a, n, x.dtype) for a, n in ((x, "x"), (W_DQ, "W_DQ"), (w_q, "w_q"), (W_UQ, "W_UQ"),
+                                           (W_DKV, "W_DKV"), (w_kv, "w_kv"), (W_UKV, "W_UKV"), (Q, "Q"),
+                                           (KC, "KC"), (kS, "kS"), (V, "V"), (cache, "cache"))],
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def mla_attn_fwd(geom: Geom, Q, KC, kS, V, g, O, maxlogit, stream=None):
+    """O <- sigmoid(g) * causal softmax(QK^T/sqrt(d_qk)) V; maxlogit[h] <- head max logit."""
+    lib = load_library()
+    torch = _torch()
+    B, T = Q.shape[0], Q.shape[1]
+    dt = _dtype_code(Q)
+    _check("mla_attn_fwd", lib.mla_attn_fwd(
+        ctypes.byref(CGeom.of(geom)), dt, B, T, _ptr(Q, "Q"), _ptr(KC, "KC", Q.dtype), _ptr(kS, "kS", Q.dtype),
+        _ptr(V, "V", Q.dtype), _ptr(g, "g", Q.dtype), _ptr(O, "O", Q.dtype), _ptr(maxlogit, "maxlogit", torch.float32),
+        _stream(stream)))
+
+
+def qkclip_rescale(geom: Geom, W_UQ, W_UKV, maxlogit, tau: float, clipped=None, gamma=None, stream=None):
+    """In-place QK-Clip of W_UQ / W_UKV for heads with maxlogit > tau."""
+    lib = load_library()
+    torch = _torch()
+    dt = _dtype_code(W_UQ)
+    _check("qkclip_rescale", lib.qkclip_rescale(
+        ctypes.byref(CGeom.of(geom)), dt, _ptr(W_UQ, "W_UQ"), _ptr(W_UKV, "W_UKV", W_UQ.dtype),
+        _ptr(maxlogit, "maxlogit", torch.float32), float(tau), _ptr(clipped, "clipped", torch.uint8),
+        _ptr(gamma, "gamma", torch.float32), _stream(stream)))
+
+
+def mla_decode_workspace(geom: Geom, dtype_code: int, n_seq: int, max_len: int) -> int:
+    return load_library().mla_decode_workspace(ctypes.byref(CGeom.of(geom)), dtype_code, n_seq, max_len)
+
+
+def mla_decode_absorbed(geom: Geom, q, W_UKV, cache, seq_offsets, max_len: int, g, O, workspace=None, stream=None):
+    """Absorbed-latent decode of one query token per sequence; see include/gmla.h."""
+    lib = load_library()
+    torch = _torch()
+    dt = _dtype_code(q)
+    n = q.shape[0]
+    need = mla_decode_workspace(geom, dt, n, max_len)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check("mla_decode_absorbed", lib.mla_decode_absorbed(
+        ctypes.byref(CGeom.of(geom)), dt, n, _ptr(q, "q"), _ptr(W_UKV, "W_UKV", q.dtype),
+        _ptr(cache, "cache", q.dtype), _ptr(seq_offsets, "seq_offsets", torch.int32), int(max_len),
+        _ptr(g, "g", q.dtype), _ptr(O, "O", q.dtype), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def mla_gemm(A, B, C, stream=None):
+    """C <- A @ B (row-major), fp32 accumulation."""
+    lib = load_library()
+    M, K = A.shape
+    N = B.shape[1]
+    _check("mla_gemm", lib.mla_gemm(_dtype_code(A), M, N, K, _ptr(A, "A"), _ptr(B, "B", A.dtype),
+                                    _ptr(C, "C", A.dtype), _stream(stream)))
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the library's device error status."""
+    return load_library().gmla_device_status(_stream(stream))
+
+
+def launch_count() -> int:
+    return int(load_library().gmla_launch_count())

@@ -1,0 +1,301 @@
+// libgmla: the C ABI declared in include/gmla.h.  One translation unit: the
+// kernel headers are included here so the device error flag and the kernels
+// live in one module.  Host code validates every argument before launching.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <atomic>
+#include <cmath>
+#include <mutex>
+
+#include "common.cuh"
+#include "simt.cuh"
+#include "clip.cuh"
+#include "sm100.cuh"
+#include "tc_attn.cuh"
+
+namespace gmla {
+
+static std::atomic<unsigned long long> g_launches{0};
+static thread_local int g_last_cuda_error = 0;
+
+void note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return GMLA_OK;
+  g_last_cuda_error = (int)e;
+  return GMLA_ECUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Validation helpers
+// ---------------------------------------------------------------------------
+static int check_geom(const gmla_geom* g) {
+  if (!g) return GMLA_EINVAL;
+  if (g->H <= 0 || g->d_model <= 0 || g->q_lora <= 0 || g->kv_lora <= 0 || g->d_c <= 0 || g->d_s < 0 ||
+      g->d_v <= 0 || !(g->rms_eps >= 0.f))
+    return GMLA_EINVAL;
+  return GMLA_OK;
+}
+static int check_dtype(gmla_dtype t) { return (t == GMLA_BF16 || t == GMLA_F32) ? GMLA_OK : GMLA_EINVAL; }
+
+#define GMLA_REQUIRE(ptr)                      \
+  do {                                         \
+    if (!(ptr)) return GMLA_EINVAL;            \
+    if (!aligned16(ptr)) return GMLA_EALIGN;   \
+  } while (0)
+#define GMLA_OPTIONAL(ptr)                           \
+  do {                                               \
+    if ((ptr) && !aligned16(ptr)) return GMLA_EALIGN; \
+  } while (0)
+#define GMLA_TRY(expr)              \
+  do {                              \
+    int _s = (expr);                \
+    if (_s != GMLA_OK) return _s;   \
+  } while (0)
+
+static inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched once through the runtime)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor [d2][d1][d0] (d0 innermost, contiguous), box {64, 128, 1},
+// 128-byte swizzle, out-of-range elements read as zero.
+static int make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
+  auto enc = get_encode();
+  if (!enc) return GMLA_EUNSUPPORTED;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GMLA_OK : GMLA_EUNSUPPORTED;
+}
+
+static bool is_k3_head_geometry(const gmla_geom* g) { return g->d_c == 128 && g->d_s == 64 && g->d_v == 128; }
+
+// ---------------------------------------------------------------------------
+// Attention forward dispatch
+// ---------------------------------------------------------------------------
+static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const void* KC, const void* kS,
+                       const void* V, const void* gate, void* O, float* maxlogit, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)tc_attn::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  CUtensorMap mQ, mKC, mKS, mV;
+  const int H = g->H;
+  GMLA_TRY(make_map_3d(&mQ, Q, (uint64_t)H * 192, T, B));
+  GMLA_TRY(make_map_3d(&mKC, KC, (uint64_t)H * 128, T, B));
+  GMLA_TRY(make_map_3d(&mKS, kS, 64, T, B));
+  GMLA_TRY(make_map_3d(&mV, V, (uint64_t)H * 128, T, B));
+  tc_attn::Params p;
+  p.B = B; p.T = T; p.H = H; p.n_qtiles = (T + tc_attn::BM - 1) / tc_attn::BM;
+  p.g = static_cast<const __nv_bfloat16*>(gate);
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.maxlogit = maxlogit;
+  p.scale = 1.f / std::sqrt(192.f);
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
+  simt::fill_kernel<<<(H + 127) / 128, 128, 0, st>>>(maxlogit, H, -INFINITY);
+  const unsigned grid = (unsigned)p.n_qtiles * (unsigned)H * (unsigned)B;
+  tc_attn::attn_fwd_kernel<<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, p);
+  note_launches(2);
+  return check_launch();
+}
+
+template <typename T>
+int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, const T* w_q,
+                        const T* W_UQ, const T* W_DKV, const T* w_kv, const T* W_UKV, T* Q, T* KC, T* kS,
+                        T* V, T* cache, void* ws, cudaStream_t st) {
+  const int M = B * Tn;
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* p = static_cast<char*>(ws);
+  T* cQ = reinterpret_cast<T*>(p);           p += al((size_t)M * g->q_lora * sizeof(T));
+  T* cQh = reinterpret_cast<T*>(p);          p += al((size_t)M * g->q_lora * sizeof(T));
+  T* ckv = reinterpret_cast<T*>(p);          p += al((size_t)M * (g->kv_lora + g->d_s) * sizeof(T));
+  T* ckvh = reinterpret_cast<T*>(p);
+  const int d_qk = g->d_c + g->d_s;
+  GMLA_TRY(simt::gemm<T>(M, g->q_lora, g->d_model, x, W_DQ, simt::EpiPlain<T>{cQ, g->q_lora}, st));
+  simt::norm_rows_kernel<T><<<M, 256, 0, st>>>(cQ, g->q_lora, w_q, g->rms_eps, cQh);
+  note_launches(1);
+  GMLA_TRY(simt::gemm<T>(M, g->H * d_qk, g->q_lora, cQh, W_UQ, simt::EpiPlain<T>{Q, g->H * d_qk}, st));
+  GMLA_TRY(simt::gemm<T>(M, g->kv_lora + g->d_s, g->d_model, x, W_DKV,
+                         simt::EpiPlain<T>{ckv, g->kv_lora + g->d_s}, st));
+  simt::norm_kv_rows_kernel<T><<<M, 256, 0, st>>>(ckv, g->kv_lora, g->d_s, w_kv, g->rms_eps, ckvh, kS, cache);
+  note_launches(1);
+  GMLA_TRY(simt::gemm<T>(M, g->H * (g->d_c + g->d_v), g->kv_lora, ckvh, W_UKV,
+                         simt::EpiSplitKV<T>{KC, V, g->H, g->d_c, g->d_v}, st));
+  return check_launch();
+}
+
+}  // namespace gmla
+
+using namespace gmla;
+
+// ===========================================================================
+// extern "C" entry points
+// ===========================================================================
+extern "C" {
+
+int gmla_version(void) { return 100; }
+
+unsigned long long gmla_launch_count(void) { return g_launches.load(); }
+
+int gmla_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* gmla_strerror(int s) {
+  switch (s) {
+    case GMLA_OK: return "ok";
+    case GMLA_EINVAL: return "invalid argument";
+    case GMLA_EALIGN: return "tensor pointer not 16-byte aligned";
+    case GMLA_EUNSUPPORTED: return "unsupported shape or dtype for this build";
+    case GMLA_ECUDA: return "CUDA error";
+    case GMLA_ETIMEOUT: return "device-side wait timed out";
+    case GMLA_EWORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int gmla_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_status(e);
+  int flag = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_status(e);
+  if (flag != 0) {
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_status(e);
+    return flag;
+  }
+  return GMLA_OK;
+}
+
+// ---------------------------------------------------------------------------
+size_t mla_up_proj_workspace(const gmla_geom* g, gmla_dtype dtype, int B, int T) {
+  if (check_geom(g) != GMLA_OK || check_dtype(dtype) != GMLA_OK || B <= 0 || T <= 0) return 0;
+  const size_t M = (size_t)B * T, es = dsize(dtype);
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return al(M * g->q_lora * es) * 2 + al(M * (g->kv_lora + g->d_s) * es) + al(M * g->kv_lora * es);
+}
+
+int mla_up_proj(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void* x, const void* W_DQ,
+                const void* w_q, const void* W_UQ, const void* W_DKV, const void* w_kv, const void* W_UKV,
+                void* Q, void* KC, void* kS, void* V, void* cache, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  if (B <= 0 || T <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(x); GMLA_REQUIRE(W_DQ); GMLA_REQUIRE(w_q); GMLA_REQUIRE(W_UQ); GMLA_REQUIRE(W_DKV);
+  GMLA_REQUIRE(w_kv); GMLA_REQUIRE(W_UKV); GMLA_REQUIRE(Q); GMLA_REQUIRE(KC); GMLA_REQUIRE(kS); GMLA_REQUIRE(V);
+  GMLA_OPTIONAL(cache);
+  if (!workspace || workspace_bytes < mla_up_proj_workspace(g, dtype, B, T)) return GMLA_EWORKSPACE;
+  if (!aligned16(workspace)) return GMLA_EALIGN;
+  cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_F32)
+    return up_proj_impl<float>(g, B, T, (const float*)x, (const float*)W_DQ, (const float*)w_q,
+                               (const float*)W_UQ, (const float*)W_DKV, (const float*)w_kv, (const float*)W_UKV,
+                               (float*)Q, (float*)KC, (float*)kS, (float*)V, (float*)cache, workspace, st);
+  using bf = __nv_bfloat16;
+  return up_proj_impl<bf>(g, B, T, (const bf*)x, (const bf*)W_DQ, (const bf*)w_q, (const bf*)W_UQ,
+                          (const bf*)W_DKV, (const bf*)w_kv, (const bf*)W_UKV, (bf*)Q, (bf*)KC, (bf*)kS, (bf*)V,
+                          (bf*)cache, workspace, st);
+}
+
+// ---------------------------------------------------------------------------
+int mla_attn_fwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void* Q, const void* KC,
+                 const void* kS, const void* V, const void* gate, void* O, float* maxlogit, void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  if (B <= 0 || T <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(Q); GMLA_REQUIRE(KC); GMLA_REQUIRE(V); GMLA_REQUIRE(O); GMLA_REQUIRE(maxlogit);
+  if (g->d_s > 0) GMLA_REQUIRE(kS);
+  GMLA_OPTIONAL(gate);
+  cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_BF16 && is_k3_head_geometry(g)) {
+    if ((long long)B * T * g->H * 192 >= (1LL << 40)) return GMLA_EUNSUPPORTED;
+    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, maxlogit, st);
+  }
+  if (g->d_c + g->d_s > 256 || g->d_v > simt::kAttnMaxDV) return GMLA_EUNSUPPORTED;
+  if (dtype == GMLA_F32)
+    return simt::attn_fwd<float>(B, T, g->H, g->d_c, g->d_s, g->d_v, (const float*)Q, (const float*)KC,
+                                 (const float*)kS, (const float*)V, (const float*)gate, (float*)O, maxlogit, st);
+  using bf = __nv_bfloat16;
+  return simt::attn_fwd<bf>(B, T, g->H, g->d_c, g->d_s, g->d_v, (const bf*)Q, (const bf*)KC, (const bf*)kS,
+                            (const bf*)V, (const bf*)gate, (bf*)O, maxlogit, st);
+}
+
+// ---------------------------------------------------------------------------
+int qkclip_rescale(const gmla_geom* g, gmla_dtype dtype, void* W_UQ, void* W_UKV, const float* maxlogit,
+                   float tau, unsigned char* clipped, float* gamma, void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  GMLA_REQUIRE(W_UQ); GMLA_REQUIRE(W_UKV);
+  if (!maxlogit) return GMLA_EINVAL;
+  if (!(tau > 0.f) || !std::isfinite(tau)) return GMLA_EINVAL;
+  cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_F32)
+    return clip::rescale<float>((float*)W_UQ, (float*)W_UKV, g->q_lora, g->kv_lora, g->H, g->d_c, g->d_s, g->d_v,
+                                maxlogit, tau, clipped, gamma, st);
+  using bf = __nv_bfloat16;
+  return clip::rescale<bf>((bf*)W_UQ, (bf*)W_UKV, g->q_lora, g->kv_lora, g->H, g->d_c, g->d_s, g->d_v, maxlogit,
+                           tau, clipped, gamma, st);
+}
+
+// ---------------------------------------------------------------------------
+size_t mla_decode_workspace(const gmla_geom* g, gmla_dtype dtype, int n_seq, int max_len) {
+  if (check_geom(g) != GMLA_OK || check_dtype(dtype) != GMLA_OK || n_seq <= 0 || max_len <= 0) return 0;
+  return simt::decode_workspace(g->H, g->kv_lora, g->d_s, n_seq, max_len);
+}
+
+int mla_decode_absorbed(const gmla_geom* g, gmla_dtype dtype, int n_seq, const void* q, const void* W_UKV,
+                        const void* cache, const int* seq_offsets, int max_len, const void* gate, void* O,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  if (n_seq <= 0 || max_len <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(q); GMLA_REQUIRE(W_UKV); GMLA_REQUIRE(cache); GMLA_REQUIRE(O);
+  if (!seq_offsets) return GMLA_EINVAL;
+  GMLA_OPTIONAL(gate);
+  if (g->kv_lora > 128 * simt::kDecMaxLatentPerThread) return GMLA_EUNSUPPORTED;
+  if (!workspace || workspace_bytes < mla_decode_workspace(g, dtype, n_seq, max_len)) return GMLA_EWORKSPACE;
+  if (!aligned16(workspace)) return GMLA_EALIGN;
+  cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_F32)
+    return simt::decode<float>(n_seq, g->H, g->d_c, g->d_s, g->d_v, g->kv_lora, (const float*)q,
+                               (const float*)W_UKV, (const float*)cache, seq_offsets, max_len, (const float*)gate,
+                               (float*)O, workspace, st);
+  using bf = __nv_bfloat16;
+  return simt::decode<bf>(n_seq, g->H, g->d_c, g->d_s, g->d_v, g->kv_lora, (const bf*)q, (const bf*)W_UKV,
+                          (const bf*)cache, seq_offsets, max_len, (const bf*)gate, (bf*)O, workspace, st);
+}
+
+// ---------------------------------------------------------------------------
+int mla_gemm(gmla_dtype dtype, int M, int N, int K, const void* A, const void* B, void* C, void* stream) {
+  GMLA_TRY(check_dtype(dtype));
+  if (M <= 0 || N <= 0 || K <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(A); GMLA_REQUIRE(B); GMLA_REQUIRE(C);
+  cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_F32)
+    return simt::gemm<float>(M, N, K, (const float*)A, (const float*)B, simt::EpiPlain<float>{(float*)C, N}, st);
+  using bf = __nv_bfloat16;
+  return simt::gemm<bf>(M, N, K, (const bf*)A, (const bf*)B, simt::EpiPlain<bf>{(bf*)C, N}, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,36 @@
+"""Helpers for the GPU parity tests (tolerances follow the acceptance bar:
+rel-L2 <= 1e-5 for fp32 outputs, <= 1e-2 for bf16 outputs, max logit within
+1e-3 relative per head, clipped-head sets and clipped weights bit-exact)."""
+import numpy as np
+
+TOL_F32 = 1e-5
+TOL_BF16 = 1e-2
+TOL_MAXLOGIT = 1e-3
+
+
+def rel_l2(got, want) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    return float(np.linalg.norm(got - want) / np.linalg.norm(want))
+
+
+def max_rel(got, want) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    return float(np.max(np.abs(got - want) / np.abs(want)))
+
+
+def dev(a, dtype, device="cuda"):
+    from gated_mla_qk_b200 import synth
+    return None if a is None else synth.to_torch(a, dtype, device)
+
+
+def host(t) -> np.ndarray:
+    import torch
+    return t.detach().to("cpu", torch.float32).numpy() if t.dtype != torch.uint8 else t.cpu().numpy()
+
+
+def check_status():
+    import gated_mla_qk_b200 as gm
+    st = gm.device_status()
+    assert st == 0, f"device status {st}"

@@ -1,0 +1,98 @@
+"""The C ABI library: it builds, loads without a GPU, exports every symbol the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gmla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_mla_qk_b200 import build
+    build.build()
+    import gated_mla_qk_b200 as g
+    return g.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b([a-z][a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if not n.startswith(("if", "defined"))))
+
+
+def test_header_declares_the_four_calls():
+    names = _declared_functions()
+    for n in ("mla_up_proj", "mla_attn_fwd", "qkclip_rescale", "mla_decode_absorbed"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    import gated_mla_qk_b200 as g
+    names = _declared_functions()
+    assert set(g.EXPORTS) <= set(names) | {"gmla_launch_count"}
+    raw = ctypes.CDLL(g.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in gmla.h but not exported"
+
+
+def test_version_and_strerror(lib):
+    assert lib.gmla_version() >= 100
+    assert lib.gmla_strerror(0) == b"ok"
+    assert lib.gmla_strerror(-5) == b"device-side wait timed out"
+    assert lib.gmla_strerror(12345) == b"unknown status"
+
+
+def _geom(g=None):
+    import gated_mla_qk_b200 as m
+    return m.CGeom.of(g or m.K3)
+
+
+def test_host_validation_without_gpu(lib):
+    import gated_mla_qk_b200 as m
+    G = ctypes.byref(_geom())
+    ok = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails earlier
+    bad = ctypes.c_void_p(0x10008)     # not 16-byte aligned
+    # null geometry, non-positive sizes, null or misaligned pointers
+    assert lib.mla_attn_fwd(None, 0, 1, 1, ok, ok, ok, ok, None, ok, ok, None) == -1
+    assert lib.mla_attn_fwd(G, 0, 0, 1, ok, ok, ok, ok, None, ok, ok, None) == -1
+    assert lib.mla_attn_fwd(G, 0, 1, 1, None, ok, ok, ok, None, ok, ok, None) == -1
+    assert lib.mla_attn_fwd(G, 0, 1, 1, bad, ok, ok, ok, None, ok, ok, None) == -2
+    assert lib.mla_attn_fwd(G, 7, 1, 1, ok, ok, ok, ok, None, ok, ok, None) == -1
+    assert lib.mla_attn_fwd(G, 0, 1, 1, ok, ok, ok, ok, bad, ok, ok, None) == -2
+    # clip: tau must be positive and finite
+    assert lib.qkclip_rescale(G, 0, ok, ok, ok, ctypes.c_float(0.0), None, None, None) == -1
+    assert lib.qkclip_rescale(G, 0, ok, ok, ok, ctypes.c_float(float("inf")), None, None, None) == -1
+    assert lib.qkclip_rescale(G, 0, ok, ok, None, ctypes.c_float(1.0), None, None, None) == -1
+    # workspace too small / missing
+    need = lib.mla_decode_workspace(G, 0, 4, 100)
+    assert need > 0
+    assert lib.mla_decode_absorbed(G, 0, 4, ok, ok, ok, ok, 100, None, ok, None, 0, None) == -6
+    assert lib.mla_decode_absorbed(G, 0, 4, ok, ok, ok, ok, 100, None, ok, ok, need - 1, None) == -6
+    assert lib.mla_decode_absorbed(G, 0, 4, ok, ok, ok, None, 100, None, ok, ok, need, None) == -1
+    assert lib.mla_decode_absorbed(G, 0, 0, ok, ok, ok, ok, 100, None, ok, ok, need, None) == -1
+    wsu = lib.mla_up_proj_workspace(G, 0, 2, 3)
+    assert wsu > 0
+    assert lib.mla_up_proj(G, 0, 2, 3, *([ok] * 11), None, ok, wsu - 1, None) == -6
+    assert lib.mla_up_proj(G, 0, 2, 3, *([ok] * 10), None, None, ok, wsu, None) == -1
+    assert lib.mla_gemm(0, 0, 4, 4, ok, ok, ok, None) == -1
+    assert lib.mla_gemm(0, 4, 4, 4, ok, bad, ok, None) == -2
+    # workspace queries reject bad sizes with 0
+    assert lib.mla_decode_workspace(G, 0, 0, 100) == 0
+    assert lib.mla_up_proj_workspace(None, 0, 1, 1) == 0
+    assert m.launch_count() == 0, "validation failures must launch nothing"
+
+
+def test_binding_refuses_missing_library(tmp_path):
+    import gated_mla_qk_b200 as m
+    saved = m._lib
+    try:
+        m._lib = None
+        with pytest.raises(ImportError):
+            m.load_library(str(tmp_path / "nope.so"))
+    finally:
+        m._lib = saved

@@ -1,0 +1,62 @@
+"""Parity of mla_decode_absorbed with the oracle (absorbed form; the oracle's
+absorbed form is itself pinned to the materialised-key form)."""
+import numpy as np
+import pytest
+
+import oracle
+from gated_mla_qk_b200 import synth
+from gpu_util import TOL_BF16, TOL_F32, check_status, dev, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(d, dtype):
+    import torch
+    import gated_mla_qk_b200 as gm
+    geom = d["geom"]
+    n = len(d["lens"])
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    O = torch.empty(n, geom.H, geom.d_v, dtype=td, device="cuda")
+    offs = torch.from_numpy(d["seq_offsets"]).cuda()
+    gm.mla_decode_absorbed(geom, dev(d["q"], dtype), dev(d["W_UKV"], dtype), dev(d["cache"], dtype), offs,
+                           int(d["lens"].max()), dev(d["g"], dtype), O)
+    check_status()
+    return host(O)
+
+
+@pytest.mark.parametrize("lens,gate", [((1, 2, 3), False), ((1, 127, 128, 129, 1000), True), ((4096, 33), False)])
+def test_small_bf16(lens, gate):
+    d = synth.decode_batch(n_seq=len(lens), lo=1, hi=2, seed=31, gate=gate)
+    # replace the drawn lengths with the listed ones (and redraw the cache to match)
+    rng = np.random.default_rng(32)
+    lens = np.array(lens)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    d.update(lens=lens, seq_offsets=offs,
+             cache=synth.round_storage(rng.standard_normal((int(offs[-1]), 576)).astype(np.float32), "bf16"))
+    got = _run(d, "bf16")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
+    assert rel_l2(got, want) <= TOL_BF16
+
+
+def test_small_fp32_tiny_geometry():
+    geom = synth.TINY
+    rng = np.random.default_rng(33)
+    lens = np.array([1, 5, 64, 300])
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    d = dict(geom=geom, lens=lens, seq_offsets=offs,
+             cache=rng.standard_normal((int(offs[-1]), geom.kv_lora + geom.d_s)).astype(np.float32),
+             q=rng.standard_normal((4, geom.H, geom.d_qk)).astype(np.float32),
+             W_UKV=(rng.standard_normal((geom.kv_lora, geom.H * (geom.d_c + geom.d_v))) / 8).astype(np.float32),
+             g=rng.standard_normal((4, geom.H * geom.d_v)).astype(np.float32))
+    got = _run(d, "f32")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], geom, d["g"])
+    assert rel_l2(got, want) <= TOL_F32
+
+
+@pytest.mark.slow
+def test_decode_64_sequences_1k_to_8k():
+    """64 sequences, lengths U[1024, 8192], 96 heads, bf16 (the decode workload)."""
+    d = synth.decode_batch()
+    got = _run(d, "bf16")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
+    assert rel_l2(got, want) <= TOL_BF16
