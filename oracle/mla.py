@@ -157,7 +157,6 @@ def attention(Q, KC, kS, V, g=None, *, heads=None, row_chunk=1024):
     Returns (O [B,T,H,d_v] float64, maxlogit [H] float64); heads not listed in
     ``heads`` are left as NaN.
     """
-    Q, KC, kS, V, g = map(_f64, (Q, KC, kS, V, g))
     B, T, H, d_qk = Q.shape
     d_v = V.shape[-1]
     scale = 1.0 / math.sqrt(d_qk)
@@ -167,20 +166,21 @@ def attention(Q, KC, kS, V, g=None, *, heads=None, row_chunk=1024):
     for h in heads:
         m_h = -np.inf
         for b in range(B):
-            K = _head_keys(KC, kS, b, h)
+            K = _f64(_head_keys(KC, kS, b, h))
+            Vh = _f64(V[b, :, h, :])
             for t0 in range(0, T, row_chunk):
                 t1 = min(T, t0 + row_chunk)
-                S = (Q[b, t0:t1, h, :] @ K[:t1].T) * scale          # [rows, t1]
+                S = (_f64(Q[b, t0:t1, h, :]) @ K[:t1].T) * scale    # [rows, t1]
                 causal = np.arange(t1)[None, :] <= np.arange(t0, t1)[:, None]
                 S = np.where(causal, S, -np.inf)
                 m_h = max(m_h, float(S.max()))
                 m = S.max(axis=1, keepdims=True)
                 P = np.exp(S - m)
                 A = P / P.sum(axis=1, keepdims=True)
-                O[b, t0:t1, h, :] = A @ V[b, :t1, h, :]
+                O[b, t0:t1, h, :] = A @ Vh[:t1]
         maxlogit[h] = m_h
     if g is not None:
-        O = O * _sigmoid(g.reshape(B, T, H, d_v))
+        O = O * _sigmoid(_f64(g).reshape(B, T, H, d_v))
     return O, maxlogit
 
 
@@ -305,17 +305,19 @@ def decode_absorbed(q, W_UKV, cache, seq_offsets, geom, g=None):
     n = q.shape[0]
     H = geom.H
     scale = 1.0 / math.sqrt(geom.d_qk)
+    W = _f64(W_UKV).reshape(geom.kv_lora, H, geom.d_c + geom.d_v)
+    W_UK = W[:, :, :geom.d_c]                      # [kv_lora, H, d_c]
+    W_UV = W[:, :, geom.d_c:]                      # [kv_lora, H, d_v]
     O = np.zeros((n, H, geom.d_v))
     for i in range(n):
-        C = cache[int(seq_offsets[i]):int(seq_offsets[i + 1])]
-        for h in range(H):
-            W_UK, W_UV = _uk_uv(W_UKV, geom, h)
-            q_abs = np.concatenate([W_UK @ q[i, h, :geom.d_c], q[i, h, geom.d_c:]])
-            s = (C @ q_abs) * scale
-            p = np.exp(s - s.max())
-            p /= p.sum()
-            u = p @ C[:, :geom.kv_lora]
-            O[i, h] = u @ W_UV
+        C = cache[int(seq_offsets[i]):int(seq_offsets[i + 1])]          # [L, kv_lora + d_s]
+        # q~_h = [q^C_h W_UK,h^T | q^S_h] for every head at once: [H, kv_lora + d_s]
+        q_abs = np.concatenate([np.einsum("lhc,hc->hl", W_UK, q[i, :, :geom.d_c]), q[i, :, geom.d_c:]], axis=-1)
+        s = (C @ q_abs.T) * scale                                         # [L, H]
+        p = np.exp(s - s.max(axis=0, keepdims=True))
+        p /= p.sum(axis=0, keepdims=True)
+        u = p.T @ C[:, :geom.kv_lora]                                     # [H, kv_lora]
+        O[i] = np.einsum("hl,lhv->hv", u, W_UV)
     if g is not None:
         O = O * _sigmoid(_f64(g).reshape(n, H, geom.d_v))
     return O
