@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--T", type=int, default=T_FWD, help="sequence length of the forward (profiling runs)")
+    ap.add_argument("--skip-decode", action="store_true", help="time the forward alone (profiling runs)")
     return ap.parse_args()
 
 
@@ -206,9 +208,11 @@ def main():
 
     # ---- inputs (seeded; each rank its own independent problem) ----
     geom = synth.K3
-    inp = synth.attn_core(B_FWD, T_FWD, geom, seed=2 + 1000 * rank, hot_heads=8, hot_scale=4.0)
+    T_run = args.T
+    fwd_flop = 2.0 * B_FWD * geom.H * T_run * (T_run + 1) / 2 * (192 + 128)
+    inp = synth.attn_core(B_FWD, T_run, geom, seed=2 + 1000 * rank, hot_heads=8, hot_scale=4.0)
     dq = {k: synth.to_torch(v, "bf16", "cuda") for k, v in inp.items()}
-    O = torch.empty(B_FWD, T_FWD, geom.H * geom.d_v, dtype=torch.bfloat16, device="cuda")
+    O = torch.empty(B_FWD, T_run, geom.H * geom.d_v, dtype=torch.bfloat16, device="cuda")
     ml = torch.empty(geom.H, dtype=torch.float32, device="cuda")
     dec = synth.decode_batch(seed=4 + 1000 * rank)
     dd = dict(q=synth.to_torch(dec["q"], "bf16", "cuda"), W_UKV=synth.to_torch(dec["W_UKV"], "bf16", "cuda"),
@@ -225,7 +229,8 @@ def main():
         gm.mla_attn_fwd(geom, dq["Q"], dq["KC"], dq["kS"], dq["V"], dq["g"], O, ml)
 
     def decode():
-        gm.mla_decode_absorbed(geom, dd["q"], dd["W_UKV"], dd["cache"], dd["offs"], max_len, None, Od, ws)
+        if not args.skip_decode:
+            gm.mla_decode_absorbed(geom, dd["q"], dd["W_UKV"], dd["cache"], dd["offs"], max_len, None, Od, ws)
 
     def step(ev):
         ev[0].record(st)
@@ -297,7 +302,7 @@ def main():
         e_ms = torch.tensor([a.elapsed_time(b) / e_steps], dtype=torch.float64, device="cuda")
         if dist is not None:
             dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * FWD_FLOP / (e_ms.item() / 1e3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": world * fwd_flop / (e_ms.item() / 1e3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms.item(),
                "what": "mla_attn_fwd with inputs copied from pinned host memory and O + maxlogit copied back"}
 
@@ -308,7 +313,7 @@ def main():
     pk = peaks()
     fwd_avg_ms = fwd_sum / args.steps
     dec_avg_ms = dec_sum / args.steps
-    fwd_tflops = FWD_FLOP / (fwd_avg_ms / 1e3) / 1e12
+    fwd_tflops = fwd_flop / (fwd_avg_ms / 1e3) / 1e12
     dec_gbs = dec_bytes / (dec_avg_ms / 1e3) / 1e9
     prof_traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
@@ -329,7 +334,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": "gated MLA attention fwd + maxlogit, B=1 T=16384 H=96 d_qk=192 d_v=128 bf16 "
                                "(heads 0-7 x4); plus absorbed decode 64 seqs L~U[1024,8192] H=96",
-                   "B": B_FWD, "T": T_FWD, "H": 96, "decode_tokens": total_tokens,
+                   "B": B_FWD, "T": T_run, "H": 96, "decode_tokens": total_tokens,
                    "l2": "inputs larger than L2 (fwd inputs 1.8 GB, decode cache %.0f MB); no flush" % (dec_bytes_cache / 1e6),
                    "parallelism": f"replicas x{world} (independent problems), maxlogit MAX all-reduce"},
         "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
@@ -347,7 +352,7 @@ def main():
     }
     if e2e:
         line["e2e"] = e2e
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and T_run == T_FWD:
         line["cpu_baseline"] = cpu_baseline(inp)
     print(json.dumps(line), flush=True)
     if dist is not None:
