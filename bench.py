@@ -194,6 +194,7 @@ def main():
     import torch
     import gated_mla_qk_b200 as gm
     from gated_mla_qk_b200 import synth
+    from gated_mla_qk_b200.dist import allreduce_maxlogit
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -236,8 +237,7 @@ def main():
         ev[0].record(st)
         fwd()
         ev[1].record(st)
-        if dist is not None:
-            dist.all_reduce(ml, op=dist.ReduceOp.MAX)
+        allreduce_maxlogit(ml)
         ev[2].record(st)
         decode()
         ev[3].record(st)
