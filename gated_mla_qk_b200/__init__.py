@@ -25,7 +25,7 @@ STATUS = {0: "GMLA_OK", -1: "GMLA_EINVAL", -2: "GMLA_EALIGN", -3: "GMLA_EUNSUPPO
           -5: "GMLA_ETIMEOUT", -6: "GMLA_EWORKSPACE"}
 
 EXPORTS = ["mla_up_proj_workspace", "mla_up_proj", "mla_attn_fwd", "qkclip_rescale", "mla_decode_workspace",
-           "mla_decode_absorbed", "mla_gemm", "gmla_device_status", "gmla_last_cuda_error", "gmla_strerror",
+           "mla_decode_absorbed", "mla_decode_absorbed_noalloc", "mla_gemm", "gmla_device_status", "gmla_last_cuda_error", "gmla_strerror",
            "gmla_version", "gmla_launch_count"]
 
 
@@ -70,6 +70,7 @@ def load_library(path: str = LIB_PATH):
         "qkclip_rescale": (I, [G, I, P, P, P, F, P, P, P]),
         "mla_decode_workspace": (S, [G, I, I, I]),
         "mla_decode_absorbed": (I, [G, I, I, P, P, P, P, I, P, P, P, S, P]),
+        "mla_decode_absorbed_noalloc": (I, [G, I, I, P, P, P, P, I, P, P, P]),
         "mla_gemm": (I, [I, I, I, I, P, P, P, P]),
         "gmla_device_status": (I, [P]),
         "gmla_last_cuda_error": (I, []),
@@ -189,6 +190,20 @@ def mla_decode_absorbed(geom: Geom, q, W_UKV, cache, seq_offsets, max_len: int, 
         _ptr(cache, "cache", q.dtype), _ptr(seq_offsets, "seq_offsets", torch.int32), int(max_len),
         _ptr(g, "g", q.dtype), _ptr(O, "O", q.dtype), _ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def mla_decode_absorbed_noalloc(geom: Geom, q, W_UKV, cache, seq_offsets, max_len: int, g, O, stream=None):
+    """mla_decode_absorbed on the library's fixed 16 MiB device scratch (no workspace).
+
+    For callers that cannot allocate device memory on their request path; see
+    include/gmla.h for the size limit and the sharing rules of the scratch.
+    """
+    lib = load_library()
+    torch = _torch()
+    _check("mla_decode_absorbed_noalloc", lib.mla_decode_absorbed_noalloc(
+        ctypes.byref(CGeom.of(geom)), _dtype_code(q), q.shape[0], _ptr(q, "q"), _ptr(W_UKV, "W_UKV", q.dtype),
+        _ptr(cache, "cache", q.dtype), _ptr(seq_offsets, "seq_offsets", torch.int32), int(max_len),
+        _ptr(g, "g", q.dtype), _ptr(O, "O", q.dtype), _stream(stream)))
 
 
 def mla_gemm(A, B, C, stream=None):

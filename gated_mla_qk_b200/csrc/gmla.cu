@@ -145,6 +145,35 @@ int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, c
   return check_launch();
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch of the non-allocating decode entry point.  The array is part
+// of the library's device image: every GPU that loads the library holds these
+// bytes until the process exits.  In host code the symbol is only a handle;
+// its device address is fetched with cudaGetSymbolAddress once per device,
+// with that device current, and cached here.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[kMaxDevices] = {};
+
+static int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= kMaxDevices) return GMLA_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return GMLA_OK;
+}
+
 }  // namespace gmla
 
 using namespace gmla;
@@ -296,6 +325,37 @@ int mla_gemm(gmla_dtype dtype, int M, int N, int K, const void* A, const void* B
     return simt::gemm<float>(M, N, K, (const float*)A, (const float*)B, simt::EpiPlain<float>{(float*)C, N}, st);
   using bf = __nv_bfloat16;
   return simt::gemm<bf>(M, N, K, (const bf*)A, (const bf*)B, simt::EpiPlain<bf>{(bf*)C, N}, st);
+}
+
+// ---------------------------------------------------------------------------
+// Decode without a caller workspace: the same kernels as the CUDA-core path of
+// mla_decode_absorbed, run on the library's fixed device scratch.  No device
+// memory is allocated; a request whose scratch need exceeds the fixed size is
+// refused with GMLA_EWORKSPACE before anything is enqueued.  Every scratch
+// byte the kernels read is written earlier in the same call, so nothing has
+// to be cleared between calls.
+int mla_decode_absorbed_noalloc(const gmla_geom* g, gmla_dtype dtype, int n_seq, const void* q,
+                                const void* W_UKV, const void* cache, const int* seq_offsets, int max_len,
+                                const void* gate, void* O, void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  if (n_seq <= 0 || max_len <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(q); GMLA_REQUIRE(W_UKV); GMLA_REQUIRE(cache); GMLA_REQUIRE(O);
+  if (!seq_offsets) return GMLA_EINVAL;
+  GMLA_OPTIONAL(gate);
+  if (g->kv_lora > 128 * simt::kDecMaxLatentPerThread) return GMLA_EUNSUPPORTED;
+  if (simt::decode_workspace(g->H, g->kv_lora, g->d_s, n_seq, max_len) > kNoAllocScratchBytes)
+    return GMLA_EWORKSPACE;
+  void* ws = nullptr;
+  GMLA_TRY(noalloc_scratch(&ws));
+  cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_F32)
+    return simt::decode<float>(n_seq, g->H, g->d_c, g->d_s, g->d_v, g->kv_lora, (const float*)q,
+                               (const float*)W_UKV, (const float*)cache, seq_offsets, max_len, (const float*)gate,
+                               (float*)O, ws, st);
+  using bf = __nv_bfloat16;
+  return simt::decode<bf>(n_seq, g->H, g->d_c, g->d_s, g->d_v, g->kv_lora, (const bf*)q, (const bf*)W_UKV,
+                          (const bf*)cache, seq_offsets, max_len, (const bf*)gate, (bf*)O, ws, st);
 }
 
 }  // extern "C"

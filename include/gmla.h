@@ -152,6 +152,37 @@ int mla_decode_absorbed(const gmla_geom* geom, gmla_dtype dtype, int n_seq,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mla_decode_absorbed_noalloc — mla_decode_absorbed for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a deployment
+ * variant.  Some callers cannot provide a workspace: a serving loop that must
+ * not call cudaMalloc / cudaFree on the request path (they can synchronise the
+ * whole device and stall other streams), or a plugin whose host framework owns
+ * every byte of device memory and hands it no scratch.  This entry point takes
+ * the same inputs and outputs as mla_decode_absorbed (minus the workspace) and
+ * runs the same CUDA-core decode kernels on a scratch array that is part of
+ * the library itself.
+ *   Limit: the call needs at most mla_decode_workspace(geom, dtype, n_seq,
+ *     max_len) bytes of scratch and the fixed array holds 16 MiB (16777216
+ *     bytes); a request that needs more returns GMLA_EWORKSPACE and enqueues
+ *     nothing.  Example: H=96, kv_lora=512 fits up to about 8 sequences of
+ *     8192 tokens.
+ *   Memory: every GPU that loads the library holds the 16 MiB until the
+ *     process exits.  No device memory is allocated by the call.
+ *   Set-up: the first call on a device (the current device) looks up the
+ *     array's device address with cudaGetSymbolAddress; make that first call
+ *     before any stream capture on that device.
+ *   Sharing: all calls on a device share the one array, which keeps the last
+ *     call's contents (nothing in it needs clearing: every byte read is first
+ *     written by the same call).  Calls that overlap on the GPU — on different
+ *     streams, or from different host threads without ordering — race on the
+ *     array and corrupt each other's results; serialise them.
+ */
+int mla_decode_absorbed_noalloc(const gmla_geom* geom, gmla_dtype dtype, int n_seq,
+                                const void* q, const void* W_UKV, const void* cache,
+                                const int* seq_offsets, int max_len, const void* g, void* O,
+                                void* stream);
+
+/*
  * mla_gemm — C[M][N] = A[M][K] B[K][N], fp32 accumulation, rounded to dtype.
  * The plain projections of the layer: the gate g = x W_g and the output
  * Delta_attn = o W_O ("Kimi K3 · Gated MLA · OpenModelAtlas", "All 20 steps").
