@@ -3,6 +3,7 @@
 // live in one module.  Host code validates every argument before launching.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <mutex>
@@ -12,6 +13,7 @@
 #include "clip.cuh"
 #include "sm100.cuh"
 #include "tc_attn.cuh"
+#include "tc_decode.cuh"
 
 namespace gmla {
 
@@ -86,7 +88,76 @@ static int make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d
   return r == CUDA_SUCCESS ? GMLA_OK : GMLA_EUNSUPPORTED;
 }
 
+// 2-D bf16 tensor [d1][d0] (d0 innermost), box {64, box1}, 128-byte swizzle.
+static int make_map_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t box1) {
+  auto enc = get_encode();
+  if (!enc) return GMLA_EUNSUPPORTED;
+  cuuint64_t dims[2] = {d0, d1};
+  cuuint64_t strides[1] = {d0 * 2};
+  cuuint32_t box[2] = {64, box1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GMLA_OK : GMLA_EUNSUPPORTED;
+}
+
 static bool is_k3_head_geometry(const gmla_geom* g) { return g->d_c == 128 && g->d_s == 64 && g->d_v == 128; }
+
+// The tensor-core decode is specialised for Kimi K3's heads and latent.
+static bool is_k3_decode_geometry(const gmla_geom* g) {
+  return is_k3_head_geometry(g) && g->H == tc_dec::HEADS && g->kv_lora == tc_dec::LAT;
+}
+
+static size_t decode_ws_bytes(const gmla_geom* g, gmla_dtype dtype, int n, int max_len) {
+  size_t b = simt::decode_workspace(g->H, g->kv_lora, g->d_s, n, max_len);
+  if (dtype == GMLA_BF16 && is_k3_decode_geometry(g)) b = std::max(b, tc_dec::workspace_bytes(n, max_len));
+  return b;
+}
+
+static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache, const int* offs, int max_len,
+                     const void* gate, void* O, void* ws, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  constexpr int kCombineSmemMax = 227 * 1024;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(tc_dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)tc_dec::SMEM_BYTES);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(tc_dec::combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kCombineSmemMax);
+  });
+  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  const int NS = tc_dec::splits(max_len);
+  if (tc_dec::combine_smem(NS) > (size_t)kCombineSmemMax) return GMLA_EUNSUPPORTED;
+  using bf = __nv_bfloat16;
+  auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
+  char* p = static_cast<char*>(ws);
+  bf* q_abs = reinterpret_cast<bf*>(p);
+  p += al((size_t)n * tc_dec::HEADS * tc_dec::WID * 2);
+  float* part_ml = reinterpret_cast<float*>(p);
+  p += al((size_t)n * NS * tc_dec::HEADS * 2 * 4);
+  float* part_u = reinterpret_cast<float*>(p);
+  CUtensorMap mQ, mC;
+  GMLA_TRY(make_map_2d(&mQ, q_abs, tc_dec::WID, (uint64_t)n * tc_dec::HEADS, tc_dec::HH));
+  // Rows of the cache map: every row a tile reads lies inside some sequence
+  // (the last tile of a chunk is shifted back to end at the chunk's end), so
+  // n * max_len bounds the coordinates that occur; rows before 0 read as zero.
+  const uint64_t rows = std::min<uint64_t>((uint64_t)n * (uint64_t)max_len, 0x7fffffffull);
+  GMLA_TRY(make_map_2d(&mC, cache, tc_dec::WID, rows, tc_dec::BT));
+  const dim3 gsm(tc_dec::HEADS, (n + 63) / 64);
+  tc_dec::absorb_kernel<<<gsm, 256, 0, st>>>(n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs);
+  tc_dec::SplitParams sp;
+  sp.n_seq = n; sp.NS = NS; sp.offs = offs;
+  sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
+  sp.part_ml = part_ml; sp.part_u = part_u;
+  tc_dec::decode_split_kernel<<<dim3(2, NS, n), 192, tc_dec::SMEM_BYTES, st>>>(mQ, mC, sp);
+  tc_dec::combine_kernel<<<gsm, 256, tc_dec::combine_smem(NS), st>>>(
+      n, NS, offs, sp.scale_log2, part_ml, part_u, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate),
+      static_cast<bf*>(O));
+  note_launches(3);
+  return check_launch();
+}
 
 // ---------------------------------------------------------------------------
 // Attention forward dispatch
@@ -290,7 +361,7 @@ int qkclip_rescale(const gmla_geom* g, gmla_dtype dtype, void* W_UQ, void* W_UKV
 // ---------------------------------------------------------------------------
 size_t mla_decode_workspace(const gmla_geom* g, gmla_dtype dtype, int n_seq, int max_len) {
   if (check_geom(g) != GMLA_OK || check_dtype(dtype) != GMLA_OK || n_seq <= 0 || max_len <= 0) return 0;
-  return simt::decode_workspace(g->H, g->kv_lora, g->d_s, n_seq, max_len);
+  return decode_ws_bytes(g, dtype, n_seq, max_len);
 }
 
 int mla_decode_absorbed(const gmla_geom* g, gmla_dtype dtype, int n_seq, const void* q, const void* W_UKV,
@@ -306,6 +377,8 @@ int mla_decode_absorbed(const gmla_geom* g, gmla_dtype dtype, int n_seq, const v
   if (!workspace || workspace_bytes < mla_decode_workspace(g, dtype, n_seq, max_len)) return GMLA_EWORKSPACE;
   if (!aligned16(workspace)) return GMLA_EALIGN;
   cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_BF16 && is_k3_decode_geometry(g))
+    return decode_tc(n_seq, q, W_UKV, cache, seq_offsets, max_len, gate, O, workspace, st);
   if (dtype == GMLA_F32)
     return simt::decode<float>(n_seq, g->H, g->d_c, g->d_s, g->d_v, g->kv_lora, (const float*)q,
                                (const float*)W_UKV, (const float*)cache, seq_offsets, max_len, (const float*)gate,

@@ -7,8 +7,8 @@
 // plus maxlogit[h] = max over b, t, s <= t of S_h[t][s] (the statistic of
 // "Anthology of the SOTA" SOTA-131's per-head max-logit check).
 //
-// One CTA = one 128-row query tile of one (batch, head); key/value tiles of
-// 128 positions stream through a 3-slot TMA ring.  The shared key k^S is
+// One CTA = one 128-row query tile of one (batch, head), launched head-major;
+// key/value tiles of 128 positions stream through a 3-slot TMA ring.  The shared key k^S is
 // never broadcast in memory: S is two MMA groups (q^C.K^C over 128 dims and
 // q^S.k^S over 64 dims) accumulating into the same TMEM tile.
 //
@@ -71,10 +71,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int HB = p.H * p.B;
-  const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / HB);   // heaviest (longest causal) tiles first
-  const int rem = (int)(blockIdx.x % HB);
-  const int h = rem % p.H, b = rem / p.H;
+  // Head-major order: the CTAs in flight work on one or two heads, whose
+  // K^C / V / k^S tiles then stay in L2 for every query tile that reads them;
+  // inside a head the longest causal rows go first.
+  const int QB = p.n_qtiles * p.B;
+  const int h = (int)(blockIdx.x / QB);
+  const int rem = (int)(blockIdx.x % QB);
+  const int qt = p.n_qtiles - 1 - rem / p.B, b = rem % p.B;
   const int n_kv = qt + 1;
 
   // A CTA launched after another one gave up does no work (the error stays
