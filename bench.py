@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--T", type=int, default=T_FWD, help="sequence length of the forward (profiling runs)")
     ap.add_argument("--skip-decode", action="store_true", help="time the forward alone (profiling runs)")
+    ap.add_argument("--skip-fwd", action="store_true", help="time the decode alone (profiling runs)")
     return ap.parse_args()
 
 
@@ -227,7 +228,8 @@ def main():
     st = torch.cuda.current_stream()
 
     def fwd():
-        gm.mla_attn_fwd(geom, dq["Q"], dq["KC"], dq["kS"], dq["V"], dq["g"], O, ml)
+        if not args.skip_fwd:
+            gm.mla_attn_fwd(geom, dq["Q"], dq["KC"], dq["kS"], dq["V"], dq["g"], O, ml)
 
     def decode():
         if not args.skip_decode:
