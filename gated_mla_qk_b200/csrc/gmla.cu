@@ -126,6 +126,9 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
     if (attr_err == cudaSuccess)
       attr_err = cudaFuncSetAttribute(tc_dec::combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       kCombineSmemMax);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(tc_dec::absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tc_dec::ABS_SMEM);
   });
   if (attr_err != cudaSuccess) return cuda_status(attr_err);
   const int NS = tc_dec::splits(max_len);
@@ -145,14 +148,15 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   // n * max_len bounds the coordinates that occur; rows before 0 read as zero.
   const uint64_t rows = std::min<uint64_t>((uint64_t)n * (uint64_t)max_len, 0x7fffffffull);
   GMLA_TRY(make_map_2d(&mC, cache, tc_dec::WID, rows, tc_dec::BT));
-  const dim3 gsm(tc_dec::HEADS, (n + 63) / 64);
-  tc_dec::absorb_kernel<<<gsm, 256, 0, st>>>(n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs);
+  tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256, tc_dec::ABS_SMEM, st>>>(
+      n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs);
   tc_dec::SplitParams sp;
   sp.n_seq = n; sp.NS = NS; sp.offs = offs;
   sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   sp.part_ml = part_ml; sp.part_u = part_u;
   tc_dec::decode_split_kernel<<<dim3(2, NS, n), 192, tc_dec::SMEM_BYTES, st>>>(mQ, mC, sp);
-  tc_dec::combine_kernel<<<gsm, 256, tc_dec::combine_smem(NS), st>>>(
+  tc_dec::combine_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::CMB_SEQ - 1) / tc_dec::CMB_SEQ), 256,
+                           tc_dec::combine_smem(NS), st>>>(
       n, NS, offs, sp.scale_log2, part_ml, part_u, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate),
       static_cast<bf*>(O));
   note_launches(3);

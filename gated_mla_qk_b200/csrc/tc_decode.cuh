@@ -47,6 +47,7 @@ constexpr uint32_t TMEM_S = 0, TMEM_U = 128;                // S^T buffers at 0 
 enum Bar { QFULL = 0, CFULL = 1, CEMPTY = 3, SFULL = 5, PFULL = 7, PVDONE = 9, DRAIN = 11, NBAR = 12 };
 
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kPrefetchAhead = 3;          // tiles brought into L2 beyond the two stages
 
 struct SplitParams {
   int n_seq, NS;
@@ -139,10 +140,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       mbar_arrive_expect_tx(bar(QFULL), NSUB * QSUB);
       for (int k = 0; k < NSUB; ++k)
         tma_load_2d(sbase + OFF_Q + k * QSUB, &tmQ, bar(QFULL), 64 * k, seq * HEADS + hh * HH);
+      // Only two 72 KB stages fit next to q~, so the tiles after them are
+      // pulled into L2 ahead of time: the stage loads then wait on L2, not HBM.
+      auto prefetch = [&](int j) {
+        if (j < nt)
+          for (int k = 0; k < NSUB; ++k) tma_prefetch_l2_2d(&tmC, 64 * k, row0 + window(j));
+      };
+      for (int j = 2; j < 2 + kPrefetchAhead; ++j) prefetch(j);
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const uint32_t st = j & 1, ph = (j >> 1) & 1;
         if (!mbar_wait(bar(CEMPTY + st), ph ^ 1u, abort)) break;
+        prefetch(j + 2 + kPrefetchAhead);
         mbar_arrive_expect_tx(bar(CFULL + st), NSUB * CSUB);
         const int r = row0 + window(j);
         for (int k = 0; k < NSUB; ++k)
@@ -167,27 +176,43 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                    idQK, (k | kk) != 0);
         mma_commit(bar(SFULL + (j & 1)));
       };
+      // Event loop: issue the score product of tile j+1 as soon as its data
+      // lands and the P.V product of tile j as soon as its P^T is written,
+      // in whichever order they become ready, so that a slow load of tile
+      // j+1 never holds back P.V of tile j (which frees a stage for loads).
       bool ok = mbar_wait(bar(QFULL), 0, abort);
       if (ok) ok = mbar_wait(bar(CFULL), 0, abort);
       if (ok) { tc_fence_after(); issue_qk(0); }
-      for (int j = 0; ok && j < nt; ++j) {
-        if (j + 1 < nt) {
-          if (!mbar_wait(bar(CFULL + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort)) break;
+      int next_qk = 1;                                  // next tile whose score product is pending
+      uint64_t t_start = 0;
+      for (int j = 0; ok && j < nt;) {
+        bool progressed = false;
+        if (next_qk < nt && next_qk <= j + 1 &&
+            mbar_try_wait(bar(CFULL + (next_qk & 1)), (next_qk >> 1) & 1)) {
           tc_fence_after();
-          issue_qk(j + 1);
+          issue_qk(next_qk++);
+          progressed = true;
         }
-        if (!mbar_wait(bar(PFULL + (j & 1)), (j >> 1) & 1, abort)) break;
-        tc_fence_after();
-        const uint32_t cst = sbase + OFF_C + (j & 1) * NSUB * CSUB;
-        const uint32_t pb = sbase + OFF_P + (j & 1) * CSUB;
+        if (next_qk > j && mbar_try_wait(bar(PFULL + (j & 1)), (j >> 1) & 1)) {
+          tc_fence_after();
+          const uint32_t cst = sbase + OFF_C + (j & 1) * NSUB * CSUB;
+          const uint32_t pb = sbase + OFF_P + (j & 1) * CSUB;
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+          for (int b = 0; b < 4; ++b)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + TMEM_U + 48u * b, sdesc_sw128(cst + (2 * b) * CSUB + kk * 2048, CSUB, 1024),
-                   sdesc_sw128(pb + kk * 2048, CSUB, 1024), idPV, (j > 0 || kk > 0));
-        mma_commit(bar(PVDONE + (j & 1)));
-        mma_commit(bar(CEMPTY + (j & 1)));
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem + TMEM_U + 48u * b, sdesc_sw128(cst + (2 * b) * CSUB + kk * 2048, CSUB, 1024),
+                     sdesc_sw128(pb + kk * 2048, CSUB, 1024), idPV, (j > 0 || kk > 0));
+          mma_commit(bar(PVDONE + (j & 1)));
+          mma_commit(bar(CEMPTY + (j & 1)));
+          ++j;
+          progressed = true;
+        }
+        if (progressed) { t_start = 0; continue; }
+        if (*abort || device_error_pending()) { *abort = 1; ok = false; break; }
+        const uint64_t now = globaltimer_ns();
+        if (t_start == 0) t_start = now;
+        else if (now - t_start > kWaitLimitNs) { raise_device_error(GMLA_ETIMEOUT); *abort = 1; ok = false; }
       }
       mma_commit(bar(DRAIN));
       mbar_wait_drain(bar(DRAIN), 0);
@@ -349,31 +374,55 @@ __device__ __forceinline__ uint32_t pack2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
   return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
 }
 
+__device__ __forceinline__ uint32_t lds32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t& r0, uint32_t& r1, const __nv_bfloat16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1) : "r"(smem_u32(p)));
+}
+
+constexpr int ABS_SEQ = 64;                    // sequences per absorb block
+constexpr int LDK = 136;                       // padded bf16 row of a 128-wide staged operand
+constexpr size_t ABS_SMEM = (size_t)(LAT + ABS_SEQ) * LDK * 2;
+
 // q~[i][h] = [q^C_h W_UK,h^T | q^S_h] in bf16.  Block = (head h, 64 sequences),
-// 8 warps; warp w computes latent columns [64w, 64w + 64).
+// 8 warps.  W_UK,h (512 x 128, one 256-byte row segment per latent index)
+// and the block's q^C rows are staged in shared memory with 16-byte loads;
+// warp w computes latent columns [64w, 64w + 64).
 __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ W_UKV,
                                                      __nv_bfloat16* __restrict__ q_abs) {
-  const int h = blockIdx.x, i0 = blockIdx.y * 64;
+  extern __shared__ __align__(16) uint8_t asm_[];
+  __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(asm_);      // [512][LDK]: W_UK,h[latent][k]
+  __nv_bfloat16* As = Ws + LAT * LDK;                               // [64][LDK]: q^C[i][k]
+  const int h = blockIdx.x, i0 = blockIdx.y * ABS_SEQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   constexpr size_t ldw = (size_t)HEADS * 256;
+  for (int e = threadIdx.x; e < LAT * 16; e += blockDim.x) {
+    const int n = e >> 4, c = e & 15;
+    cp_async16(Ws + n * LDK + c * 8, W_UKV + (size_t)n * ldw + (size_t)h * 256 + c * 8);
+  }
+  for (int e = threadIdx.x; e < ABS_SEQ * 16; e += blockDim.x) {
+    const int r = e >> 4, c = e & 15, i = i0 + r;
+    if (i < n_seq) cp_async16(As + r * LDK + c * 8, q + ((size_t)i * HEADS + h) * 192 + c * 8);
+    else *reinterpret_cast<uint4*>(As + r * LDK + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_wait_all();
+  __syncthreads();
 #pragma unroll 1
-  for (int mt = 0; mt < 4; ++mt) {
-    const int ra = i0 + mt * 16 + g, rb = ra + 8;
+  for (int mt = 0; mt < ABS_SEQ / 16; ++mt) {
     float acc[8][4] = {};
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      uint32_t a[4] = {0u, 0u, 0u, 0u};
       const int k0 = kk * 16 + 2 * t;
-      if (ra < n_seq) { const __nv_bfloat16* qa = q + ((size_t)ra * HEADS + h) * 192; a[0] = ld_u32(qa + k0); a[2] = ld_u32(qa + k0 + 8); }
-      if (rb < n_seq) { const __nv_bfloat16* qb = q + ((size_t)rb * HEADS + h) * 192; a[1] = ld_u32(qb + k0); a[3] = ld_u32(qb + k0 + 8); }
+      const __nv_bfloat16* ar = As + (mt * 16 + g) * LDK + k0;
+      const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDK), lds32(ar + 8), lds32(ar + 8 * LDK + 8)};
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
-        const int n = warp * 64 + nt * 8 + g;
-        const __nv_bfloat16* wr = W_UKV + (size_t)n * ldw + (size_t)h * 256;
-        mma16816(acc[nt], a, ld_u32(wr + k0), ld_u32(wr + k0 + 8));
+        const __nv_bfloat16* br = Ws + (warp * 64 + nt * 8 + g) * LDK + k0;
+        mma16816(acc[nt], a, lds32(br), lds32(br + 8));
       }
     }
+    const int ra = i0 + mt * 16 + g, rb = ra + 8;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
       const int col = warp * 64 + nt * 8 + 2 * t;
@@ -383,83 +432,107 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
         *reinterpret_cast<__nv_bfloat162*>(q_abs + ((size_t)rb * HEADS + h) * WID + col) = __floats2bfloat162_rn(acc[nt][2], acc[nt][3]);
     }
   }
-  // q^S passes through unchanged.
-  for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
-    const int ii = i0 + e / 64, c = e % 64;
-    if (ii < n_seq) q_abs[((size_t)ii * HEADS + h) * WID + LAT + c] = q[((size_t)ii * HEADS + h) * 192 + 128 + c];
+  // q^S passes through unchanged: 64 values = 8 x 16 bytes per sequence.
+  for (int e = threadIdx.x; e < ABS_SEQ * 8; e += blockDim.x) {
+    const int i = i0 + (e >> 3), c = e & 7;
+    if (i < n_seq)
+      *reinterpret_cast<uint4*>(q_abs + ((size_t)i * HEADS + h) * WID + LAT + c * 8) =
+          *reinterpret_cast<const uint4*>(q + ((size_t)i * HEADS + h) * 192 + 128 + c * 8);
   }
 }
 
+constexpr int CMB_SEQ = 32;                    // sequences per combine block
+constexpr int LDU = LAT + 8;                   // padded bf16 row of the merged latent tile
+
 // Merge the chunks of each sequence for head h, normalise, and project with
-// W_UV,h.  Block = (head h, 64 sequences), 8 warps; warp w owns output
-// columns [16w, 16w + 16).
+// W_UV,h.  Block = (head h, 32 sequences), 8 warps; warp w owns output
+// columns [16w, 16w + 16).  W_UV,h (512 x 128, row-major) is staged in shared
+// memory and fed to the MMA through transposing matrix loads.
 __global__ void __launch_bounds__(256) combine_kernel(int n_seq, int NS, const int* __restrict__ offs, float scale_log2,
                                                       const float* __restrict__ part_ml, const float* __restrict__ part_u,
                                                       const __nv_bfloat16* __restrict__ W_UKV,
                                                       const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ O) {
-  constexpr int LDA = LAT + 8;                          // padded row (bf16) of the merged latent tile
   extern __shared__ __align__(16) uint8_t csm[];
-  __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(csm);   // [64][LDA]
-  float* wsc = reinterpret_cast<float*>(csm + 64 * LDA * 2);   // [64][CHUNK splits] weights
-  const int h = blockIdx.x, i0 = blockIdx.y * 64;
+  __nv_bfloat16* Wv = reinterpret_cast<__nv_bfloat16*>(csm);                    // [512][LDK]
+  __nv_bfloat16* U = Wv + LAT * LDK;                                             // [32][LDU]
+  float* wsc = reinterpret_cast<float*>(U + CMB_SEQ * LDU);                      // [32][NS]
+  int* nsv = reinterpret_cast<int*>(wsc + CMB_SEQ * NS);                         // [32]
+  const int h = blockIdx.x, i0 = blockIdx.y * CMB_SEQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t = lane & 3;
-  // 1) merge weights per (sequence, chunk): w_s = 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c)
-  if (threadIdx.x < 64) {
-    const int i = i0 + threadIdx.x;
+  constexpr size_t ldw = (size_t)HEADS * 256;
+  for (int e = threadIdx.x; e < LAT * 16; e += blockDim.x) {
+    const int k = e >> 4, c = e & 15;
+    cp_async16(Wv + k * LDK + c * 8, W_UKV + (size_t)k * ldw + (size_t)h * 256 + 128 + c * 8);
+  }
+  // merge weights per (sequence, chunk): w_s = 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c)
+  if (threadIdx.x < CMB_SEQ) {
+    const int r = threadIdx.x, i = i0 + r;
+    int ns = 0;
     if (i < n_seq) {
-      const int ns = min(NS, (offs[i + 1] - offs[i] + CHUNK - 1) / CHUNK);
+      ns = min(NS, (offs[i + 1] - offs[i] + CHUNK - 1) / CHUNK);
       float M = -INFINITY;
       for (int s = 0; s < ns; ++s) M = fmaxf(M, part_ml[(((size_t)i * NS + s) * HEADS + h) * 2]);
       float Ls = 0.f;
       for (int s = 0; s < ns; ++s) {
         const size_t k = (((size_t)i * NS + s) * HEADS + h) * 2;
         const float w = ex2((part_ml[k] - M) * scale_log2);
-        wsc[threadIdx.x * NS + s] = w;
+        wsc[r * NS + s] = w;
         Ls += part_ml[k + 1] * w;
       }
       const float inv = 1.f / Ls;
-      for (int s = 0; s < ns; ++s) wsc[threadIdx.x * NS + s] *= inv;
-      for (int s = ns; s < NS; ++s) wsc[threadIdx.x * NS + s] = 0.f;
-    } else {
-      for (int s = 0; s < NS; ++s) wsc[threadIdx.x * NS + s] = 0.f;
+      for (int s = 0; s < ns; ++s) wsc[r * NS + s] *= inv;
     }
+    nsv[r] = ns;
   }
   __syncthreads();
-  // 2) merged, normalised latent u[i][:] in bf16
-  for (int e = threadIdx.x; e < 64 * LAT; e += blockDim.x) {
-    const int ii = e / LAT, l = e % LAT, i = i0 + ii;
-    float u = 0.f;
-    if (i < n_seq) {
-      const int ns = min(NS, (offs[i + 1] - offs[i] + CHUNK - 1) / CHUNK);
-      for (int s = 0; s < ns; ++s) u += part_u[(((size_t)i * NS + s) * HEADS + h) * LAT + l] * wsc[ii * NS + s];
+  // merged, normalised latent u[i][:] in bf16: each thread owns 16 groups of
+  // four latents (rows r = tid/128 + 2k); the chunk loop is outermost so the
+  // 16 loads of one chunk are independent and in flight together.
+  constexpr int PER = CMB_SEQ * (LAT / 4) / 256;
+  float4 u[PER];
+  int maxns = 0;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) { u[k] = make_float4(0.f, 0.f, 0.f, 0.f); maxns = max(maxns, nsv[(threadIdx.x + 256 * k) / (LAT / 4)]); }
+  for (int s = 0; s < maxns; ++s) {
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int e = threadIdx.x + 256 * k, r = e / (LAT / 4), l = (e % (LAT / 4)) * 4, i = i0 + r;
+      if (s < nsv[r]) {
+        const float w = wsc[r * NS + s];
+        const float4 v = *reinterpret_cast<const float4*>(part_u + (((size_t)i * NS + s) * HEADS + h) * LAT + l);
+        u[k].x = fmaf(v.x, w, u[k].x); u[k].y = fmaf(v.y, w, u[k].y);
+        u[k].z = fmaf(v.z, w, u[k].z); u[k].w = fmaf(v.w, w, u[k].w);
+      }
     }
-    A[ii * LDA + l] = __float2bfloat16_rn(u);
   }
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int e = threadIdx.x + 256 * k, r = e / (LAT / 4), l = (e % (LAT / 4)) * 4;
+    __nv_bfloat162* d = reinterpret_cast<__nv_bfloat162*>(U + r * LDU + l);
+    d[0] = __floats2bfloat162_rn(u[k].x, u[k].y);
+    d[1] = __floats2bfloat162_rn(u[k].z, u[k].w);
+  }
+  cp_async_wait_all();
   __syncthreads();
-  // 3) O[i][h][:] = u W_UV,h  (K = 512, N = 128)
-  constexpr size_t ldw = (size_t)HEADS * 256;
-  const __nv_bfloat16* Wv = W_UKV + (size_t)h * 256 + 128;
-  float acc[4][2][4] = {};
+  // O[i][h][:] = u W_UV,h  (M = 32 sequences, N = 128, K = 512)
+  float acc[2][2][4] = {};
 #pragma unroll 4
   for (int kk = 0; kk < LAT / 16; ++kk) {
-    const int k0 = kk * 16 + 2 * t;
+    const int k0 = kk * 16;
     uint32_t bf[2][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int n = warp * 16 + nt * 8 + gq;
-      bf[nt][0] = pack2(Wv[(size_t)k0 * ldw + n], Wv[(size_t)(k0 + 1) * ldw + n]);
-      bf[nt][1] = pack2(Wv[(size_t)(k0 + 8) * ldw + n], Wv[(size_t)(k0 + 9) * ldw + n]);
-    }
+    for (int nt = 0; nt < 2; ++nt)
+      ldsm_x2_trans(bf[nt][0], bf[nt][1], Wv + (k0 + (lane & 15)) * LDK + warp * 16 + nt * 8);
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
-      const __nv_bfloat16* ar = A + (mt * 16 + gq) * LDA + k0;
-      uint32_t a[4] = {ld_u32(ar), ld_u32(ar + 8 * LDA), ld_u32(ar + 8), ld_u32(ar + 8 * LDA + 8)};
+    for (int mt = 0; mt < 2; ++mt) {
+      const __nv_bfloat16* ar = U + (mt * 16 + gq) * LDU + k0 + 2 * t;
+      const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDU), lds32(ar + 8), lds32(ar + 8 * LDU + 8)};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) mma16816(acc[mt][nt], a, bf[nt][0], bf[nt][1]);
     }
   }
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -478,7 +551,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int n_seq, int NS, const i
       }
 }
 
-inline size_t combine_smem(int NS) { return 64 * (LAT + 8) * 2 + 64 * (size_t)NS * 4; }
+inline size_t combine_smem(int NS) { return (size_t)LAT * LDK * 2 + (size_t)CMB_SEQ * LDU * 2 + (size_t)CMB_SEQ * NS * 4 + CMB_SEQ * 4; }
 
 inline int splits(int max_len) { return (max_len + CHUNK - 1) / CHUNK; }
 
