@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cmath>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "simt.cuh"
@@ -14,6 +15,7 @@
 #include "sm100.cuh"
 #include "tc_attn.cuh"
 #include "tc_decode.cuh"
+#include "tc_gemm.cuh"
 
 namespace gmla {
 
@@ -195,6 +197,34 @@ static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const vo
   return check_launch();
 }
 
+// bf16 GEMM on the tensor cores when the shapes suit TMA (row strides of
+// whole 16-byte units), else the CUDA-core GEMM.  mode 1 writes the per-head
+// [K^C_h | V_h] split of an N = H * 256 product.
+static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfloat16* B, __nv_bfloat16* C,
+                     __nv_bfloat16* KC, __nv_bfloat16* V, int H, int d_c, int d_v, int mode, cudaStream_t st) {
+  const bool tc = (K % 8 == 0) && (N % 8 == 0) && (mode == 0 || (d_c == 128 && d_v == 128));
+  if (!tc) {
+    if (mode == 1) return simt::gemm<__nv_bfloat16>(M, N, K, A, B, simt::EpiSplitKV<__nv_bfloat16>{KC, V, H, d_c, d_v}, st);
+    return simt::gemm<__nv_bfloat16>(M, N, K, A, B, simt::EpiPlain<__nv_bfloat16>{C, N}, st);
+  }
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(tc_gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)tc_gemm::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  CUtensorMap mA, mB;
+  GMLA_TRY(make_map_2d(&mA, A, (uint64_t)K, (uint64_t)M, tc_gemm::BM));
+  GMLA_TRY(make_map_2d(&mB, B, (uint64_t)N, (uint64_t)K, tc_gemm::BK));
+  tc_gemm::Params p;
+  p.M = M; p.N = N; p.K = K; p.C = C; p.KC = KC; p.V = V; p.H = H; p.mode = mode;
+  const unsigned grid = (unsigned)((N + tc_gemm::BN - 1) / tc_gemm::BN) * (unsigned)((M + tc_gemm::BM - 1) / tc_gemm::BM);
+  tc_gemm::gemm_kernel<<<grid, 192, tc_gemm::SMEM_BYTES, st>>>(mA, mB, p);
+  note_launches(1);
+  return check_launch();
+}
+
 template <typename T>
 int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, const T* w_q,
                         const T* W_UQ, const T* W_DKV, const T* w_kv, const T* W_UKV, T* Q, T* KC, T* kS,
@@ -207,16 +237,25 @@ int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, c
   T* ckv = reinterpret_cast<T*>(p);          p += al((size_t)M * (g->kv_lora + g->d_s) * sizeof(T));
   T* ckvh = reinterpret_cast<T*>(p);
   const int d_qk = g->d_c + g->d_s;
-  GMLA_TRY(simt::gemm<T>(M, g->q_lora, g->d_model, x, W_DQ, simt::EpiPlain<T>{cQ, g->q_lora}, st));
+  auto plain = [&](int Mm, int N, int K, const T* A, const T* B, T* C) -> int {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value)
+      return gemm_bf16(Mm, N, K, A, B, C, nullptr, nullptr, 0, 0, 0, 0, st);
+    else
+      return simt::gemm<T>(Mm, N, K, A, B, simt::EpiPlain<T>{C, N}, st);
+  };
+  GMLA_TRY(plain(M, g->q_lora, g->d_model, x, W_DQ, cQ));
   simt::norm_rows_kernel<T><<<M, 256, 0, st>>>(cQ, g->q_lora, w_q, g->rms_eps, cQh);
   note_launches(1);
-  GMLA_TRY(simt::gemm<T>(M, g->H * d_qk, g->q_lora, cQh, W_UQ, simt::EpiPlain<T>{Q, g->H * d_qk}, st));
-  GMLA_TRY(simt::gemm<T>(M, g->kv_lora + g->d_s, g->d_model, x, W_DKV,
-                         simt::EpiPlain<T>{ckv, g->kv_lora + g->d_s}, st));
+  GMLA_TRY(plain(M, g->H * d_qk, g->q_lora, cQh, W_UQ, Q));
+  GMLA_TRY(plain(M, g->kv_lora + g->d_s, g->d_model, x, W_DKV, ckv));
   simt::norm_kv_rows_kernel<T><<<M, 256, 0, st>>>(ckv, g->kv_lora, g->d_s, w_kv, g->rms_eps, ckvh, kS, cache);
   note_launches(1);
-  GMLA_TRY(simt::gemm<T>(M, g->H * (g->d_c + g->d_v), g->kv_lora, ckvh, W_UKV,
-                         simt::EpiSplitKV<T>{KC, V, g->H, g->d_c, g->d_v}, st));
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    GMLA_TRY(gemm_bf16(M, g->H * (g->d_c + g->d_v), g->kv_lora, ckvh, W_UKV, nullptr, KC, V, g->H, g->d_c, g->d_v, 1, st));
+  } else {
+    GMLA_TRY(simt::gemm<T>(M, g->H * (g->d_c + g->d_v), g->kv_lora, ckvh, W_UKV,
+                           simt::EpiSplitKV<T>{KC, V, g->H, g->d_c, g->d_v}, st));
+  }
   return check_launch();
 }
 
@@ -401,7 +440,7 @@ int mla_gemm(gmla_dtype dtype, int M, int N, int K, const void* A, const void* B
   if (dtype == GMLA_F32)
     return simt::gemm<float>(M, N, K, (const float*)A, (const float*)B, simt::EpiPlain<float>{(float*)C, N}, st);
   using bf = __nv_bfloat16;
-  return simt::gemm<bf>(M, N, K, (const bf*)A, (const bf*)B, simt::EpiPlain<bf>{(bf*)C, N}, st);
+  return gemm_bf16(M, N, K, (const bf*)A, (const bf*)B, (bf*)C, nullptr, nullptr, 0, 0, 0, 0, st);
 }
 
 // ---------------------------------------------------------------------------

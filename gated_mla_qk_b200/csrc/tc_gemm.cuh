@@ -1,0 +1,147 @@
+// bf16 GEMM on the 5th-generation tensor cores for the low-rank projections
+// of the layer ("Kimi K3 · Gated MLA · OpenModelAtlas", "All 20 steps":
+// c^Q = x W_DQ, q = c^Q W_UQ, [c^KV k^S] = x W_DKV, [k^C v] = c^KV W_UKV).
+//
+// C[M][N] = A[M][K] B[K][N], all row-major; fp32 accumulation in TMEM.
+// One CTA per 128 x 256 output tile.  A tiles (128 x 64, K-major) and B tiles
+// (64 x 256, N contiguous = MN-major) stream through a 4-stage TMA ring; one
+// thread issues tcgen05.mma (M=128, N=256, K=16) into a 256-column TMEM
+// accumulator; four epilogue warps read it back with tcgen05.ld and store
+// bf16.  The epilogue either writes C row-major or, for the key/value
+// up-projection, splits each 256-column tile (= one head) into K^C and V.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace gmla {
+namespace tc_gemm {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 64, NSTAGE = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2;                 // 16 KB
+constexpr uint32_t BSUB = BK * 128;                       // one 64 (k) x 64 (n) sub-tile, 8 KB
+constexpr uint32_t B_BYTES = 4 * BSUB;                    // 32 KB
+constexpr uint32_t STAGE = A_BYTES + B_BYTES;             // 48 KB
+constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
+
+enum Bar { FULL = 0, EMPTY = NSTAGE, ACC = 2 * NSTAGE, NBAR = 2 * NSTAGE + 1 };
+
+struct Params {
+  int M, N, K;
+  __nv_bfloat16* C;          // [M][N] (mode 0)
+  __nv_bfloat16* KC;         // [M][H][128] (mode 1)
+  __nv_bfloat16* V;          // [M][H][128] (mode 1)
+  int H;
+  int mode;                  // 0: plain, 1: per-head split of [K^C_h | V_h] (N = H * 256)
+};
+
+__global__ void __launch_bounds__(192, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  volatile int* abort = &abort_flag;
+  auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int tn = blockIdx.x % n_tiles, tm = blockIdx.x / n_tiles;
+  const int nk = (p.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) abort_flag = device_error_pending() ? 1 : 0;
+  __syncthreads();
+  if (abort_flag) return;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) { tmem_alloc(smem_u32(&tmem_slot), 256); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
+      int issued = 0;
+      for (int k = 0; k < nk; ++k) {
+        const uint32_t s = k % NSTAGE, ph = (k / NSTAGE) & 1;
+        if (!mbar_wait(bar(EMPTY + s), ph ^ 1u, abort)) break;
+        const uint32_t st = sbase + s * STAGE;
+        mbar_arrive_expect_tx(bar(FULL + s), STAGE);
+        tma_load_2d(st, &tmA, bar(FULL + s), k * BK, tm * BM);
+        for (int c = 0; c < 4; ++c) tma_load_2d(st + A_BYTES + c * BSUB, &tmB, bar(FULL + s), tn * BN + 64 * c, k * BK);
+        ++issued;
+      }
+      for (int k = (issued > NSTAGE ? issued - NSTAGE : 0); k < issued; ++k)
+        mbar_wait_drain(bar(FULL + k % NSTAGE), (k / NSTAGE) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);   // A K-major, B MN-major
+      for (int k = 0; k < nk; ++k) {
+        const uint32_t s = k % NSTAGE, ph = (k / NSTAGE) & 1;
+        if (!mbar_wait(bar(FULL + s), ph, abort)) break;
+        tc_fence_after();
+        const uint32_t st = sbase + s * STAGE;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_ss(tmem, sdesc_sw128(st + kk * 32, 16, 1024), sdesc_sw128(st + A_BYTES + kk * 2048, BSUB, 1024), idesc,
+                 (k > 0 || kk > 0));
+        mma_commit(bar(EMPTY + s));
+      }
+      mma_commit(bar(ACC));
+      mbar_wait_drain(bar(ACC), 0);
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) .. + 31
+    const int sub = warp & 3;
+    const int row = tm * BM + sub * 32 + lane;
+    const bool ok = mbar_wait(bar(ACC), 0, abort);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + 32u * c, v);
+        tmem_wait_ld();
+        const int col0 = tn * BN + 32 * c;
+        if (row < p.M && col0 < p.N) {
+          __nv_bfloat16* dst;
+          if (p.mode == 1) {
+            const int h = col0 / 256, j = col0 % 256;
+            dst = (j < 128) ? p.KC + ((size_t)row * p.H + h) * 128 + j : p.V + ((size_t)row * p.H + h) * 128 + (j - 128);
+          } else {
+            dst = p.C + (size_t)row * p.N + col0;
+          }
+          if (col0 + 32 <= p.N) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              d4[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                 pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (col0 + e < p.N) dst[e] = __float2bfloat16_rn(v[e]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace tc_gemm
+}  // namespace gmla
