@@ -1,12 +1,16 @@
 #!/usr/bin/env python
 """Throughput of the gated MLA hot path on B200.
 
-One step = one causal gated attention forward with the fused per-head max
-logit on the long-context workload (B=1, T=16384, H=96, d_qk=192, d_v=128,
-bf16, heads 0-7 x4), plus one absorbed-latent decode of 64 sequences with
-context lengths U[1024, 8192] over the 576-wide latent cache.  ``value`` is
-the forward's TFLOP/s (causal half including the diagonal: 2*B*H*T(T+1)/2*320
-FLOP per call); the decode's HBM GB/s is reported beside it.
+One step = one pass of the whole hot path on three synthetic workloads:
+  * the QK-Clip chain at Kimi K3 size (x[4,4096,7168], bf16): up-projections,
+    attention forward + per-head max logit, QK-Clip at tau = 100, and the
+    recompute (up-projections + forward) with the clipped weights;
+  * the causal gated attention forward with the fused max logit on the
+    long-context workload (B=1, T=16384, H=96, d_qk=192, d_v=128, heads 0-7 x4);
+  * the absorbed-latent decode of 64 sequences, context lengths U[1024, 8192].
+``value`` is the long-context forward's TFLOP/s (causal half including the
+diagonal: 2*B*H*T(T+1)/2*320 FLOP per call); every other part is reported
+beside it with its own roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -47,6 +51,7 @@ def parse():
     ap.add_argument("--T", type=int, default=T_FWD, help="sequence length of the forward (profiling runs)")
     ap.add_argument("--skip-decode", action="store_true", help="time the forward alone (profiling runs)")
     ap.add_argument("--skip-fwd", action="store_true", help="time the decode alone (profiling runs)")
+    ap.add_argument("--skip-clip", action="store_true", help="leave out the K3 QK-Clip chain (profiling runs)")
     return ap.parse_args()
 
 
@@ -227,6 +232,44 @@ def main():
     dec_bytes = dec_bytes_cache + 2 * 512 * 96 * 128 * 2 + 64 * 96 * (192 + 128) * 2
     st = torch.cuda.current_stream()
 
+    # ---- QK-Clip chain at K3 size ----
+    chain = None
+    if not args.skip_clip:
+        L = synth.k3_clip_layer(seed=3 + 1000 * rank)
+        Bc, Tc = L["x"].shape[:2]
+        bf = torch.bfloat16
+        chain = dict(
+            x=synth.to_torch(L["x"], "bf16", "cuda"),
+            W={k: synth.to_torch(L[k], "bf16", "cuda") for k in ("W_DQ", "w_q", "W_UQ", "W_DKV", "w_kv", "W_UKV")},
+            Q=torch.empty(Bc, Tc, 96, 192, dtype=bf, device="cuda"), KC=torch.empty(Bc, Tc, 96, 128, dtype=bf, device="cuda"),
+            kS=torch.empty(Bc, Tc, 64, dtype=bf, device="cuda"), V=torch.empty(Bc, Tc, 96, 128, dtype=bf, device="cuda"),
+            O=torch.empty(Bc, Tc, 96 * 128, dtype=bf, device="cuda"), ml=torch.empty(96, dtype=torch.float32, device="cuda"),
+            clipped=torch.empty(96, dtype=torch.uint8, device="cuda"), tau=L["tau"], B=Bc, T=Tc)
+        chain["WQ"] = chain["W"]["W_UQ"].clone()
+        chain["WKV"] = chain["W"]["W_UKV"].clone()
+        chain["ws"] = torch.empty(gm.mla_up_proj_workspace(geom, gm.GMLA_BF16, Bc, Tc), dtype=torch.uint8, device="cuda")
+        del L
+    UP_FLOP = 2.0 * 4 * 4096 * (7168 * 1536 + 1536 * 18432 + 7168 * 576 + 512 * 24576)
+    C3_FLOP = 2.0 * 4 * 96 * 4096 * 4097 / 2 * 320
+
+    def clip_chain(ev):
+        c = chain
+        c["WQ"].copy_(c["W"]["W_UQ"]); c["WKV"].copy_(c["W"]["W_UKV"])     # pristine weights each step
+        W = c["W"]
+
+        def up():
+            gm.mla_up_proj(geom, c["x"], W["W_DQ"], W["w_q"], c["WQ"], W["W_DKV"], W["w_kv"], c["WKV"], c["Q"], c["KC"],
+                           c["kS"], c["V"], None, c["ws"])
+
+        def att():
+            gm.mla_attn_fwd(geom, c["Q"], c["KC"], c["kS"], c["V"], None, c["O"], c["ml"])
+
+        ev[0].record(st); up(); ev[1].record(st); att()
+        allreduce_maxlogit(c["ml"])
+        ev[2].record(st)
+        gm.qkclip_rescale(geom, c["WQ"], c["WKV"], c["ml"], c["tau"], c["clipped"], None)
+        ev[3].record(st); up(); ev[4].record(st); att(); ev[5].record(st)
+
     def fwd():
         if not args.skip_fwd:
             gm.mla_attn_fwd(geom, dq["Q"], dq["KC"], dq["kS"], dq["V"], dq["g"], O, ml)
@@ -236,6 +279,8 @@ def main():
             gm.mla_decode_absorbed(geom, dd["q"], dd["W_UKV"], dd["cache"], dd["offs"], max_len, None, Od, ws)
 
     def step(ev):
+        if chain is not None:
+            clip_chain(ev[4:])
         ev[0].record(st)
         fwd()
         ev[1].record(st)
@@ -244,11 +289,12 @@ def main():
         decode()
         ev[3].record(st)
 
+    warm_ev = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
     for _ in range(args.warmup):
-        fwd(); decode()
+        step(warm_ev)
     torch.cuda.synchronize()
     assert gm.device_status() == 0
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(args.steps)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -268,10 +314,16 @@ def main():
     total_ms = start.elapsed_time(end)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    t = torch.tensor([total_ms, sum(fwd_ms), sum(dec_ms)], dtype=torch.float64, device="cuda")
+    parts = [sum(fwd_ms), sum(dec_ms)]
+    if chain is not None:
+        parts += [sum(e[4].elapsed_time(e[5]) + e[7].elapsed_time(e[8]) for e in evs),      # up-projections (x2)
+                  sum(e[5].elapsed_time(e[6]) + e[8].elapsed_time(e[9]) for e in evs),      # K3 forwards (x2)
+                  sum(e[6].elapsed_time(e[7]) for e in evs)]                                 # QK-Clip
+    t = torch.tensor([total_ms] + parts, dtype=torch.float64, device="cuda")
     if dist is not None:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_sum, dec_sum = t.tolist()
+    total_ms, fwd_sum, dec_sum, *chain_sums = t.tolist()
+    n_clipped = int(chain["clipped"].sum().item()) if chain is not None else 0
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
@@ -335,7 +387,8 @@ def main():
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": "gated MLA attention fwd + maxlogit, B=1 T=16384 H=96 d_qk=192 d_v=128 bf16 "
-                               "(heads 0-7 x4); plus absorbed decode 64 seqs L~U[1024,8192] H=96",
+                               "(heads 0-7 x4); plus the K3 QK-Clip chain x[4,4096,7168] (up-proj, fwd, clip, "
+                               "recompute) and absorbed decode 64 seqs L~U[1024,8192] H=96",
                    "B": B_FWD, "T": T_run, "H": 96, "decode_tokens": total_tokens,
                    "l2": "inputs larger than L2 (fwd inputs 1.8 GB, decode cache %.0f MB); no flush" % (dec_bytes_cache / 1e6),
                    "parallelism": f"replicas x{world} (independent problems), maxlogit MAX all-reduce"},
@@ -348,10 +401,29 @@ def main():
                    "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": pk["hbm"], "unit": "GB/s",
                                 "frac": dec_gbs / pk["hbm"]}},
         "fwd_ms": fwd_avg_ms,
+        "parts": {},
         "gpu_launches": launches,
         "device_status": status,
         "clocks": clk.summary(),
     }
+    if chain is not None:
+        up_ms = chain_sums[0] / (2 * args.steps)
+        c3_ms = chain_sums[1] / (2 * args.steps)
+        clip_ms = chain_sums[2] / args.steps
+        clip_bytes = 2 * n_clipped * (1536 * 128 + 1536 * 64 + 512 * 128) * 2
+        line["parts"] = {
+            "up_proj_B4_T4096": {"ms": up_ms, "value": UP_FLOP / (up_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                                 "roofline": {"bound": "tensor", "peak": pk["bf16"],
+                                              "frac": UP_FLOP / (up_ms / 1e3) / 1e12 / pk["bf16"]}},
+            "attn_fwd_B4_T4096_nogate": {"ms": c3_ms, "value": C3_FLOP / (c3_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                                         "roofline": {"bound": "tensor", "peak": pk["bf16"],
+                                                      "frac": C3_FLOP / (c3_ms / 1e3) / 1e12 / pk["bf16"]}},
+            "qkclip": {"ms": clip_ms, "clipped_heads": n_clipped, "bytes": clip_bytes,
+                       "value": clip_bytes / (clip_ms / 1e3) / 1e9, "unit": "GB/s",
+                       "roofline": {"bound": "hbm", "peak": pk["hbm"], "frac": clip_bytes / (clip_ms / 1e3) / 1e9 / pk["hbm"]}},
+        }
+    line["parts"]["attn_fwd_B1_T16384"] = {"ms": fwd_avg_ms, "value": fwd_tflops, "unit": "TFLOP/s"}
+    line["parts"]["decode_64seq"] = {"ms": dec_avg_ms, "value": dec_gbs, "unit": "GB/s"}
     if e2e:
         line["e2e"] = e2e
     if not args.no_cpu_baseline and T_run == T_FWD:
