@@ -143,8 +143,7 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   float* part_ml = reinterpret_cast<float*>(p);
   p += al((size_t)n * NS * tc_dec::HEADS * 2 * 4);
   float* part_u = reinterpret_cast<float*>(p);
-  CUtensorMap mQ, mC;
-  GMLA_TRY(make_map_2d(&mQ, q_abs, tc_dec::WID, (uint64_t)n * tc_dec::HEADS, tc_dec::HH));
+  CUtensorMap mC;
   // Rows of the cache map: every row a tile reads lies inside some sequence
   // (the last tile of a chunk is shifted back to end at the chunk's end), so
   // n * max_len bounds the coordinates that occur; rows before 0 read as zero.
@@ -153,10 +152,10 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256, tc_dec::ABS_SMEM, st>>>(
       n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs);
   tc_dec::SplitParams sp;
-  sp.n_seq = n; sp.NS = NS; sp.offs = offs;
+  sp.n_seq = n; sp.NS = NS; sp.offs = offs; sp.q_abs = q_abs;
   sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   sp.part_ml = part_ml; sp.part_u = part_u;
-  tc_dec::decode_split_kernel<<<dim3(2, NS, n), 192, tc_dec::SMEM_BYTES, st>>>(mQ, mC, sp);
+  tc_dec::decode_split_kernel<<<dim3(2, NS, n), 192, tc_dec::SMEM_BYTES, st>>>(mC, sp);
   tc_dec::combine_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::CMB_SEQ - 1) / tc_dec::CMB_SEQ), 256,
                            tc_dec::combine_smem(NS), st>>>(
       n, NS, offs, sp.scale_log2, part_ml, part_u, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate),

@@ -11,16 +11,18 @@
 //   o_h  = (u_h / l) W_UV,h  (* sigmoid(g))                  (combine kernel)
 //
 // Split kernel: one CTA per (sequence, 1024-token chunk, half of the heads).
-// The latent cache streams through two 72 KB TMA stages in tiles of 64
-// tokens.  Per tile, two tcgen05 products share the same 128B-swizzled tile:
-//   S^T [64 tokens x 48 heads] = cache_tile (K-major, K = 576) x q~^T
-//   U^T [512 latent x 48 heads] += cache_tile^T (MN-major) x P^T
-// so the cache is read from HBM once and never transposed.  Softmax runs per
-// head, i.e. down a TMEM column (across token lanes), with a lazily updated
-// per-head reference max: a cross-lane max is only taken when some logit
-// exceeds the reference by more than 2^8 (always on a chunk's first tile).
-// Each CTA writes its partial (reference max, sum, U) in fp32; the combine
-// kernel merges the chunks of a sequence and applies W_UV.
+// Heads sit on the MMA's M side (48 heads as an M = 64 tile, half the TMEM
+// lanes), tokens on N:
+//   S [48 heads x 64 tokens] = q~ (A, resident in TMEM) x cache_tile^T (B, K-major)
+//   U [48 heads x 512]      += P (A, smem) x cache_tile (B, MN-major)
+// so the 64-token tile of the latent cache, streamed through three 72 KB TMA
+// stages, is the only operand read from shared memory by the score product,
+// and the same 128B-swizzled tile serves both products.  q~ and S live in the
+// upper half of each TMEM sub-partition, U in the lower half.  Softmax is per
+// row (one head per thread) with a lazily updated reference max; a row of U
+// is rescaled only when its max grows by more than 2^8, and only while no
+// product of this CTA is in flight.  Each CTA writes its partial (reference
+// max, sum, U) in fp32; the combine kernel merges the chunks and applies W_UV.
 #pragma once
 
 #include "sm100.cuh"
@@ -30,80 +32,43 @@ namespace tc_dec {
 
 using namespace sm100;
 
-constexpr int HEADS = 96, HH = 48;        // heads, heads per CTA
-constexpr int BT = 64;                     // tokens per tile
+constexpr int HEADS = 96, HH = 48;        // heads, heads per CTA (an M = 64 tile with 16 idle rows)
+constexpr int BT = 64;                     // tokens per tile (N of the score product)
 constexpr int CHUNK = 1024;                // tokens per split (work item)
-constexpr int LAT = 512, WID = 576, NSUB = 9;
-constexpr uint32_t QSUB = HH * 128;        // one [48 x 64] bf16 sub-tile of q~ (6 KB)
-constexpr uint32_t CSUB = BT * 128;        // one [64 x 64] bf16 sub-tile of the cache (8 KB)
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_C = OFF_Q + NSUB * QSUB;             // 2 stages x 9 sub-tiles
-constexpr uint32_t OFF_P = OFF_C + 2 * NSUB * CSUB;         // 2 P^T buffers [64 tokens x 128 B]
-constexpr uint32_t OFF_RED = OFF_P + 2 * CSUB;              // float scratch for reductions
-constexpr uint32_t OFF_BAR = OFF_RED + 2048;
+constexpr int LAT = 512, WID = 576, NSUB = 9, NSTAGE = 3;
+constexpr uint32_t CSUB = BT * 128;        // one [64 tokens x 64] bf16 sub-tile of the cache (8 KB)
+constexpr uint32_t STAGE = NSUB * CSUB;    // 72 KB
+constexpr uint32_t OFF_C = 0;
+constexpr uint32_t OFF_P = OFF_C + NSTAGE * STAGE;          // P [64 head rows x 128 B]
+constexpr uint32_t OFF_BAR = OFF_P + CSUB;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t TMEM_S = 0, TMEM_U = 128;                // S^T buffers at 0 and 64; U^T blocks at 128 + 48b
+// TMEM columns.  Upper lanes (0-15 of each sub-partition): q~ as the A operand
+// (576 bf16 = 288 columns) and two S buffers; lower lanes (16-31): U.
+constexpr uint32_t TM_Q = 0, TM_S = 288, TM_U = 0;
+constexpr uint32_t LANE_LO = 16u << 16;   // lane offset of the lower half
 
-enum Bar { QFULL = 0, CFULL = 1, CEMPTY = 3, SFULL = 5, PFULL = 7, PVDONE = 9, DRAIN = 11, NBAR = 12 };
+enum Bar { CFULL = 0, CEMPTY = CFULL + NSTAGE, SFULL = CEMPTY + NSTAGE, PFULL = SFULL + 2, PVDONE = PFULL + 1,
+           QREADY = PVDONE + 1, DRAIN = QREADY + 1, NBAR = DRAIN + 1 };
 
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kPrefetchAhead = 3;          // tiles brought into L2 beyond the two stages
+constexpr int kPrefetchAhead = 2;          // tiles brought into L2 beyond the stages
 
 struct SplitParams {
   int n_seq, NS;
-  const int* offs;          // [n_seq + 1]
-  float scale_log2;         // log2(e) / sqrt(192)
-  float* part_ml;           // [n][NS][96][2]: reference max (raw logit units), sum
-  float* part_u;            // [n][NS][96][512]
+  const int* offs;                 // [n_seq + 1]
+  const __nv_bfloat16* q_abs;      // [n][96][576]
+  float scale_log2;                // log2(e) / sqrt(192)
+  float* part_ml;                  // [n][NS][96][2]: reference max (raw logit units), sum
+  float* part_u;                   // [n][NS][96][512]
 };
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])),
-        "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
-      : "memory");
-}
-// 48 consecutive TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld48(uint32_t taddr, float (&v)[48]) {
-  tmem_ld16(taddr, v);
-  tmem_ld16(taddr + 16, v + 16);
-  tmem_ld16(taddr + 32, v + 32);
-}
-__device__ __forceinline__ void tmem_st48(uint32_t taddr, const float (&v)[48]) {
-  tmem_st16(taddr, v);
-  tmem_st16(taddr + 16, v + 16);
-  tmem_st16(taddr + 32, v + 32);
-}
-// Named barrier over the four softmax warps only.
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
 __global__ void __launch_bounds__(192, 1)
-decode_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC, SplitParams p) {
+decode_split_kernel(const __grid_constant__ CUtensorMap tmC, SplitParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
-  float* red = reinterpret_cast<float*>(smem_raw + (sbase - sraw) + OFF_RED);   // [4][48] + m[48] + corr[48] + flags
-  float* sm_m = red + 4 * HH;
-  float* sm_corr = sm_m + HH;
-  int* sm_flag = reinterpret_cast<int*>(sm_corr + HH);
   volatile int* abort = &abort_flag;
   auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
 
@@ -120,91 +85,78 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   __syncthreads();
   if (abort_flag) return;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == PFULL || i == PFULL + 1) ? 128 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == PFULL || i == QREADY) ? 128 : 1);
     fence_mbar_init();
   }
-  if (threadIdx.x < HH) sm_m[threadIdx.x] = -INFINITY;
   if (warp == 5) { tmem_alloc(smem_u32(&tmem_slot), 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
-  // Window of tile j inside the chunk: rows [ws, ws + 64) relative to row0,
-  // shifted back for the last tile so that no row past the chunk's end is read.
+  // Rows [ws, ws + 64) of tile j relative to row0; the last tile is shifted
+  // back so that no row past the chunk's end is read.
   auto window = [&](int j) { return min(j * BT, len - BT); };
 
   if (warp == 4) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmC);
-      mbar_arrive_expect_tx(bar(QFULL), NSUB * QSUB);
-      for (int k = 0; k < NSUB; ++k)
-        tma_load_2d(sbase + OFF_Q + k * QSUB, &tmQ, bar(QFULL), 64 * k, seq * HEADS + hh * HH);
-      // Only two 72 KB stages fit next to q~, so the tiles after them are
-      // pulled into L2 ahead of time: the stage loads then wait on L2, not HBM.
+      tma_prefetch_desc(&tmC);
       auto prefetch = [&](int j) {
         if (j < nt)
           for (int k = 0; k < NSUB; ++k) tma_prefetch_l2_2d(&tmC, 64 * k, row0 + window(j));
       };
-      for (int j = 2; j < 2 + kPrefetchAhead; ++j) prefetch(j);
+      for (int j = NSTAGE; j < NSTAGE + kPrefetchAhead; ++j) prefetch(j);
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
-        const uint32_t st = j & 1, ph = (j >> 1) & 1;
+        const uint32_t st = j % NSTAGE, ph = (j / NSTAGE) & 1;
         if (!mbar_wait(bar(CEMPTY + st), ph ^ 1u, abort)) break;
-        prefetch(j + 2 + kPrefetchAhead);
-        mbar_arrive_expect_tx(bar(CFULL + st), NSUB * CSUB);
+        prefetch(j + NSTAGE + kPrefetchAhead);
+        mbar_arrive_expect_tx(bar(CFULL + st), STAGE);
         const int r = row0 + window(j);
         for (int k = 0; k < NSUB; ++k)
-          tma_load_2d(sbase + OFF_C + st * NSUB * CSUB + k * CSUB, &tmC, bar(CFULL + st), 64 * k, r);
+          tma_load_2d(sbase + OFF_C + st * STAGE + k * CSUB, &tmC, bar(CFULL + st), 64 * k, r);
         ++issued;
       }
-      mbar_wait_drain(bar(QFULL), 0);
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) mbar_wait_drain(bar(CFULL + (j & 1)), (j >> 1) & 1);
+      for (int j = (issued > NSTAGE ? issued - NSTAGE : 0); j < issued; ++j)
+        mbar_wait_drain(bar(CFULL + j % NSTAGE), (j / NSTAGE) & 1);
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      constexpr uint32_t idQK = idesc_bf16_f32(64, HH, false, false);   // cache (K-major) x q~ (K-major)
-      constexpr uint32_t idPV = idesc_bf16_f32(128, HH, true, true);    // cache^T (MN-major) x P^T (MN-major)
+      constexpr uint32_t idQK = idesc_bf16_f32(64, BT, false, false);    // q~ (TMEM) x cache tile (K-major)
+      constexpr uint32_t idPV = idesc_bf16_f32(64, 256, false, true);    // P (K-major) x cache tile (MN-major)
       auto issue_qk = [&](int j) {
-        const uint32_t cst = sbase + OFF_C + (j & 1) * NSUB * CSUB;
-        const uint32_t d = tmem + TMEM_S + (uint32_t)(j & 1) * 64u;
+        const uint32_t cst = sbase + OFF_C + (j % NSTAGE) * STAGE;
+        const uint32_t d = tmem + TM_S + (uint32_t)(j & 1) * 64u;
 #pragma unroll
-        for (int k = 0; k < NSUB; ++k)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(d, sdesc_sw128(cst + k * CSUB + kk * 32, 16, 1024), sdesc_sw128(sbase + OFF_Q + k * QSUB + kk * 32, 16, 1024),
-                   idQK, (k | kk) != 0);
+        for (int i = 0; i < 4 * NSUB; ++i)
+          mma_ts(d, tmem + TM_Q + 8u * i, sdesc_sw128(cst + (i >> 2) * CSUB + (i & 3) * 32, 16, 1024), idQK, i != 0);
         mma_commit(bar(SFULL + (j & 1)));
       };
-      // Event loop: issue the score product of tile j+1 as soon as its data
-      // lands and the P.V product of tile j as soon as its P^T is written,
-      // in whichever order they become ready, so that a slow load of tile
-      // j+1 never holds back P.V of tile j (which frees a stage for loads).
-      bool ok = mbar_wait(bar(QFULL), 0, abort);
-      if (ok) ok = mbar_wait(bar(CFULL), 0, abort);
-      if (ok) { tc_fence_after(); issue_qk(0); }
-      int next_qk = 1;                                  // next tile whose score product is pending
+      // Event loop: issue the score product of a tile as soon as its data has
+      // landed (and its S buffer is free), and the P.V product of tile j as
+      // soon as P is written, in whichever order they become ready.
+      bool ok = mbar_wait(bar(QREADY), 0, abort);
+      int next_qk = 0;
       uint64_t t_start = 0;
       for (int j = 0; ok && j < nt;) {
         bool progressed = false;
         if (next_qk < nt && next_qk <= j + 1 &&
-            mbar_try_wait(bar(CFULL + (next_qk & 1)), (next_qk >> 1) & 1)) {
+            mbar_try_wait(bar(CFULL + next_qk % NSTAGE), (next_qk / NSTAGE) & 1)) {
           tc_fence_after();
           issue_qk(next_qk++);
           progressed = true;
         }
-        if (next_qk > j && mbar_try_wait(bar(PFULL + (j & 1)), (j >> 1) & 1)) {
+        if (next_qk > j && mbar_try_wait(bar(PFULL), j & 1)) {
           tc_fence_after();
-          const uint32_t cst = sbase + OFF_C + (j & 1) * NSUB * CSUB;
-          const uint32_t pb = sbase + OFF_P + (j & 1) * CSUB;
+          const uint32_t cst = sbase + OFF_C + (j % NSTAGE) * STAGE;
 #pragma unroll
-          for (int b = 0; b < 4; ++b)
+          for (int kk = 0; kk < BT / 16; ++kk)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ss(tmem + TMEM_U + 48u * b, sdesc_sw128(cst + (2 * b) * CSUB + kk * 2048, CSUB, 1024),
-                     sdesc_sw128(pb + kk * 2048, CSUB, 1024), idPV, (j > 0 || kk > 0));
-          mma_commit(bar(PVDONE + (j & 1)));
-          mma_commit(bar(CEMPTY + (j & 1)));
+            for (int nh = 0; nh < 2; ++nh)
+              mma_ss(tmem + LANE_LO + TM_U + 256u * nh, sdesc_sw128(sbase + OFF_P + kk * 32, 16, 1024),
+                     sdesc_sw128(cst + (4 * nh) * CSUB + kk * 2048, CSUB, 1024), idPV, (j > 0 || kk > 0));
+          mma_commit(bar(PVDONE));
+          mma_commit(bar(CEMPTY + j % NSTAGE));
           ++j;
           progressed = true;
         }
@@ -220,134 +172,121 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax (warps 0-3)
+    // Lanes 0-15 of warp w own head rows 16w + lane (upper TMEM lanes: q~, S);
+    // lanes 16-31 hold the U rows of the same heads (lower TMEM lanes).
     const float c = p.scale_log2;
-    const float thr_add = kRescaleLog2 / c;             // reference max may lag the true max by this much
+    const float thr_add = kRescaleLog2 / c;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int r = warp * 16 + lane;                     // token row of this thread (lanes 0-15)
-    float lsum[HH];
+    const bool upper = lane < 16;
+    const int hr = warp * 16 + (lane & 15);              // head row inside the CTA (valid if < 48)
+    const bool head_ok = hr < HH;
+    // Load q~ into the upper TMEM lanes (the lower lanes write zeros into the
+    // U columns, which the first P.V product overwrites).
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + ((size_t)seq * HEADS + hh * HH + (head_ok ? hr : 0)) * WID);
+#pragma unroll 1
+      for (int cch = 0; cch < 9; ++cch) {
+        float v[32];
 #pragma unroll
-    for (int h = 0; h < HH; ++h) lsum[h] = 0.f;
-    // A failed (timed-out) wait turns `ok` off for the rest of the kernel; the
-    // four warps still walk through every named barrier below in the same
-    // order (they never leave the loop), so none is left waiting at one.
+        for (int q = 0; q < 8; ++q) {
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (upper && head_ok) x = src[cch * 8 + q];
+          v[4 * q + 0] = __uint_as_float(x.x); v[4 * q + 1] = __uint_as_float(x.y);
+          v[4 * q + 2] = __uint_as_float(x.z); v[4 * q + 3] = __uint_as_float(x.w);
+        }
+        tmem_st32(tmem + lane_off + TM_Q + 32u * cch, v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(QREADY));
+    }
+    float m_used = -INFINITY, lsum = 0.f;
     bool ok = true;
     auto wait_warp = [&](int i, uint32_t ph) {
       const bool w = ok && mbar_wait(bar(i), ph, abort);
       ok = __all_sync(0xffffffffu, w) != 0;
       return ok;
     };
-    for (int j = 0; j < nt; ++j) {
-      float s[HH];
-      if (wait_warp(SFULL + (j & 1), (j >> 1) & 1)) {
-        tc_fence_after();
-        tmem_ld48(tmem + lane_off + TMEM_S + (uint32_t)(j & 1) * 64u, s);
-        tmem_wait_ld();
-      }
+    for (int j = 0; j < nt && ok; ++j) {
+      if (!wait_warp(SFULL + (j & 1), (j >> 1) & 1)) break;
+      tc_fence_after();
+      float s[BT];
+      tmem_ld32(tmem + lane_off + TM_S + (uint32_t)(j & 1) * 64u, *reinterpret_cast<float(*)[32]>(&s[0]));
+      tmem_ld32(tmem + lane_off + TM_S + (uint32_t)(j & 1) * 64u + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
+      tmem_wait_ld();
       const int ws = window(j);
-      const int tok = ws + r;                            // token index inside the chunk
-      const bool valid = ok && lane < 16 && tok >= j * BT && tok < len;
-      bool ex = false;
+      float mx = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < HH; ++h) {
-        s[h] = valid ? s[h] : -INFINITY;
-        ex |= s[h] > sm_m[h] + thr_add;
+      for (int k = 0; k < BT; ++k) {
+        const int tok = ws + k;
+        s[k] = (upper && tok >= j * BT && tok < len) ? s[k] : -INFINITY;
+        mx = fmaxf(mx, s[k]);
       }
-      const int vote = __any_sync(0xffffffffu, ex);
-      if (lane == 0) sm_flag[warp] = vote;
-      softmax_sync();
-      const bool any = (sm_flag[0] | sm_flag[1] | sm_flag[2] | sm_flag[3]) != 0;
-      softmax_sync();                                    // flags read before they are rewritten
-      if (any) {
-        // Exact per-head max of this tile (down the token lanes), then move
-        // the reference of every head whose new logits passed it.
-#pragma unroll
-        for (int h = 0; h < HH; ++h) {
-          float v = s[h];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) red[warp * HH + h] = v;
-        }
-        softmax_sync();
-        if (threadIdx.x < HH) {
-          const int h = threadIdx.x;
-          const float tmax = fmaxf(fmaxf(red[h], red[HH + h]), fmaxf(red[2 * HH + h], red[3 * HH + h]));
-          const float m_old = sm_m[h];
-          const float m_new = (tmax > m_old + thr_add) ? tmax : m_old;
-          sm_corr[h] = (m_new == m_old) ? 1.f : ex2((m_old - m_new) * c);
-          sm_m[h] = m_new;
-        }
-        softmax_sync();
-        // U must hold every product issued so far before it is rescaled.
-        if (j > 0 && wait_warp(PVDONE + ((j - 1) & 1), ((j - 1) >> 1) & 1)) {
-          tc_fence_after();
+      const bool need = upper && head_ok && mx > m_used + thr_add;     // first tile: m_used = -inf
+      const float m_new = need ? mx : m_used;
+      const float corr = need ? ex2((m_used - m_new) * c) : 1.f;       // 0 on the first tile
+      // P buffer and U: the previous product must have finished.
+      if (j > 0 && !wait_warp(PVDONE, (j - 1) & 1)) break;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // Rare: rescale this warp's U rows.  No product of this CTA is in
+        // flight once the score product of tile j+1 (if issued) is done,
+        // because P.V of tile j waits for this warp's arrival below.
+        if (j + 1 < nt && !wait_warp(SFULL + ((j + 1) & 1), ((j + 1) >> 1) & 1)) break;
+        tc_fence_after();
+        const float f = __shfl_sync(0xffffffffu, corr, lane & 15);   // lower lane takes its head's factor
 #pragma unroll 1
-          for (int b = 0; b < 4; ++b) {
-            float u[HH];
-            const uint32_t ua = tmem + lane_off + TMEM_U + 48u * b;
-            tmem_ld48(ua, u);
-            tmem_wait_ld();
+        for (int cch = 0; cch < LAT / 32; ++cch) {
+          float u[32];
+          tmem_ld32(tmem + lane_off + TM_U + 32u * cch, u);
+          tmem_wait_ld();
+          if (!upper) {
 #pragma unroll
-            for (int h = 0; h < HH; ++h) u[h] *= sm_corr[h];
-            tmem_st48(ua, u);
+            for (int e = 0; e < 32; ++e) u[e] *= f;
           }
-          tmem_wait_st();
+          tmem_st32(tmem + lane_off + TM_U + 32u * cch, u);
         }
-#pragma unroll
-        for (int h = 0; h < HH; ++h) lsum[h] *= sm_corr[h];
+        tmem_wait_st();
       }
-      // P^T buffer (j & 1) was last read by the product of tile j - 2.
-      const bool pfree = (j < 2) ? ok : wait_warp(PVDONE + (j & 1), ((j - 2) >> 1) & 1);
-      if (pfree && lane < 16) {
-        const uint32_t prow = sbase + OFF_P + (uint32_t)(j & 1) * CSUB + (uint32_t)r * 128u;
+      lsum *= corr;
+      m_used = m_new;
+      if (upper) {
+        // Rows of the 16 idle heads (48-63) get P = 0.
+        const float neg = head_ok ? -m_used * c : 0.f;
+        const uint32_t prow = sbase + OFF_P + (uint32_t)hr * 128u;
 #pragma unroll
-        for (int cc = 0; cc < HH / 8; ++cc) {
+        for (int cc = 0; cc < 8; ++cc) {
           float e[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const int h = cc * 8 + q;
-            e[q] = ex2(fmaf(s[h], c, -sm_m[h] * c));
-            lsum[h] += e[q];
+            e[q] = head_ok ? ex2(fmaf(s[8 * cc + q], c, neg)) : 0.f;
+            lsum += e[q];
           }
-          st_shared_v4(prow + ((uint32_t)(cc ^ (r & 7)) << 4), pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
+          st_shared_v4(prow + ((uint32_t)(cc ^ (hr & 7)) << 4), pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
                        pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
         }
       }
-      if (ok) {
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(bar(PFULL + (j & 1)));
-      }
-      softmax_sync();                                    // sm_m is reused by the next tile
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(PFULL));
     }
-    const bool done = wait_warp(PVDONE + ((nt - 1) & 1), ((nt - 1) >> 1) & 1);
-    tc_fence_after();
-    // Sum of the exponentials per head over every token lane.
-#pragma unroll
-    for (int h = 0; h < HH; ++h) {
-      float v = lsum[h];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) red[warp * HH + h] = v;
-    }
-    softmax_sync();
-    const int all_done = (int)done;
-    if (lane == 0) sm_flag[warp] = all_done;
-    softmax_sync();
-    if (sm_flag[0] & sm_flag[1] & sm_flag[2] & sm_flag[3]) {
+    if (ok && wait_warp(PVDONE, (nt - 1) & 1)) {
+      tc_fence_after();
       const size_t pbase = ((size_t)seq * p.NS + split) * HEADS + hh * HH;
-      if (threadIdx.x < HH) {
-        const int h = threadIdx.x;
-        p.part_ml[(pbase + h) * 2 + 0] = sm_m[h];
-        p.part_ml[(pbase + h) * 2 + 1] = red[h] + red[HH + h] + red[2 * HH + h] + red[3 * HH + h];
+      if (upper && head_ok) {
+        p.part_ml[(pbase + hr) * 2 + 0] = m_used;
+        p.part_ml[(pbase + hr) * 2 + 1] = lsum;
       }
+      float* dst = p.part_u + (pbase + (head_ok ? hr : 0)) * LAT;
 #pragma unroll 1
-      for (int b = 0; b < 4; ++b) {
-        float u[HH];
-        tmem_ld48(tmem + lane_off + TMEM_U + 48u * b, u);
+      for (int cch = 0; cch < LAT / 32; ++cch) {
+        float u[32];
+        tmem_ld32(tmem + lane_off + TM_U + 32u * cch, u);
         tmem_wait_ld();
-        const int l = 128 * b + warp * 32 + lane;        // latent index of this lane
+        if (!upper && head_ok) {
+          float4* d4 = reinterpret_cast<float4*>(dst + 32 * cch);
 #pragma unroll
-        for (int h = 0; h < HH; ++h) p.part_u[(pbase + h) * LAT + l] = u[h];
+          for (int q = 0; q < 8; ++q) d4[q] = make_float4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+        }
       }
     }
   }
