@@ -121,20 +121,18 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
                      const void* gate, void* O, void* ws, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
-  constexpr int kCombineSmemMax = 227 * 1024;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(tc_dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)tc_dec::SMEM_BYTES);
     if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(tc_dec::combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      kCombineSmemMax);
+      attr_err = cudaFuncSetAttribute(tc_dec::project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tc_dec::PRJ_SMEM);
     if (attr_err == cudaSuccess)
       attr_err = cudaFuncSetAttribute(tc_dec::absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)tc_dec::ABS_SMEM);
   });
   if (attr_err != cudaSuccess) return cuda_status(attr_err);
   const int NS = tc_dec::splits(max_len);
-  if (tc_dec::combine_smem(NS) > (size_t)kCombineSmemMax) return GMLA_EUNSUPPORTED;
   using bf = __nv_bfloat16;
   auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
   char* p = static_cast<char*>(ws);
@@ -143,6 +141,8 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   float* part_ml = reinterpret_cast<float*>(p);
   p += al((size_t)n * NS * tc_dec::HEADS * 2 * 4);
   float* part_u = reinterpret_cast<float*>(p);
+  p += al((size_t)n * NS * tc_dec::HEADS * tc_dec::LAT * 4);
+  bf* u_merged = reinterpret_cast<bf*>(p);
   CUtensorMap mC;
   // Rows of the cache map: every row a tile reads lies inside some sequence
   // (the last tile of a chunk is shifted back to end at the chunk's end), so
@@ -156,11 +156,10 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   sp.part_ml = part_ml; sp.part_u = part_u;
   tc_dec::decode_split_kernel<<<dim3(2, NS, n), 192, tc_dec::SMEM_BYTES, st>>>(mC, sp);
-  tc_dec::combine_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::CMB_SEQ - 1) / tc_dec::CMB_SEQ), 256,
-                           tc_dec::combine_smem(NS), st>>>(
-      n, NS, offs, sp.scale_log2, part_ml, part_u, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate),
-      static_cast<bf*>(O));
-  note_launches(3);
+  tc_dec::merge_kernel<<<(n * tc_dec::HEADS + 7) / 8, 256, 0, st>>>(n, NS, offs, sp.scale_log2, part_ml, part_u, u_merged);
+  tc_dec::project_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::PRJ_SEQ - 1) / tc_dec::PRJ_SEQ), 256, tc_dec::PRJ_SMEM, st>>>(
+      n, u_merged, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate), static_cast<bf*>(O));
+  note_launches(4);
   return check_launch();
 }
 

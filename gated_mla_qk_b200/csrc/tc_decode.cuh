@@ -380,81 +380,72 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
   }
 }
 
-constexpr int CMB_SEQ = 32;                    // sequences per combine block
-constexpr int LDU = LAT + 8;                   // padded bf16 row of the merged latent tile
+// Merge the chunks of each (sequence, head): one warp per pair, 16 latents per
+// lane.  u = sum_s U_s 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c), in bf16.
+__global__ void __launch_bounds__(256) merge_kernel(int n_seq, int NS, const int* __restrict__ offs, float scale_log2,
+                                                    const float* __restrict__ part_ml, const float* __restrict__ part_u,
+                                                    __nv_bfloat16* __restrict__ u_out) {
+  const int pair = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (pair >= n_seq * HEADS) return;
+  const int i = pair / HEADS, h = pair % HEADS;
+  const int ns = min(NS, (offs[i + 1] - offs[i] + CHUNK - 1) / CHUNK);
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, part_ml[(((size_t)i * NS + s) * HEADS + h) * 2]);
+  float4 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float Ls = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const size_t k = ((size_t)i * NS + s) * HEADS + h;
+    const float w = ex2((part_ml[2 * k] - M) * scale_log2);
+    Ls += part_ml[2 * k + 1] * w;
+    const float4* src = reinterpret_cast<const float4*>(part_u + k * LAT);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = src[lane + 32 * q];
+      acc[q].x = fmaf(v.x, w, acc[q].x); acc[q].y = fmaf(v.y, w, acc[q].y);
+      acc[q].z = fmaf(v.z, w, acc[q].z); acc[q].w = fmaf(v.w, w, acc[q].w);
+    }
+  }
+  const float inv = 1.f / Ls;
+  __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(u_out + ((size_t)i * HEADS + h) * LAT);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int l4 = lane + 32 * q;
+    dst[2 * l4] = __floats2bfloat162_rn(acc[q].x * inv, acc[q].y * inv);
+    dst[2 * l4 + 1] = __floats2bfloat162_rn(acc[q].z * inv, acc[q].w * inv);
+  }
+}
 
-// Merge the chunks of each sequence for head h, normalise, and project with
-// W_UV,h.  Block = (head h, 32 sequences), 8 warps; warp w owns output
-// columns [16w, 16w + 16).  W_UV,h (512 x 128, row-major) is staged in shared
-// memory and fed to the MMA through transposing matrix loads.
-__global__ void __launch_bounds__(256) combine_kernel(int n_seq, int NS, const int* __restrict__ offs, float scale_log2,
-                                                      const float* __restrict__ part_ml, const float* __restrict__ part_u,
+constexpr int PRJ_SEQ = 64;                    // sequences per projection block
+constexpr int LDU = LAT + 8;                   // padded bf16 row of the staged latent tile
+constexpr size_t PRJ_SMEM = (size_t)LAT * LDK * 2 + (size_t)PRJ_SEQ * LDU * 2;
+
+// o[i][h] = u[i][h] W_UV,h (* sigmoid(g)).  Block = (head h, 64 sequences),
+// 8 warps; warp w owns output columns [16w, 16w + 16).  W_UV,h (512 x 128,
+// row-major) and the block's merged latents are staged with cp.async; W_UV,h
+// feeds the MMA through transposing matrix loads.
+__global__ void __launch_bounds__(256) project_kernel(int n_seq, const __nv_bfloat16* __restrict__ u_in,
                                                       const __nv_bfloat16* __restrict__ W_UKV,
                                                       const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ O) {
   extern __shared__ __align__(16) uint8_t csm[];
   __nv_bfloat16* Wv = reinterpret_cast<__nv_bfloat16*>(csm);                    // [512][LDK]
-  __nv_bfloat16* U = Wv + LAT * LDK;                                             // [32][LDU]
-  float* wsc = reinterpret_cast<float*>(U + CMB_SEQ * LDU);                      // [32][NS]
-  int* nsv = reinterpret_cast<int*>(wsc + CMB_SEQ * NS);                         // [32]
-  const int h = blockIdx.x, i0 = blockIdx.y * CMB_SEQ;
+  __nv_bfloat16* U = Wv + LAT * LDK;                                             // [64][LDU]
+  const int h = blockIdx.x, i0 = blockIdx.y * PRJ_SEQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t = lane & 3;
   constexpr size_t ldw = (size_t)HEADS * 256;
   for (int e = threadIdx.x; e < LAT * 16; e += blockDim.x) {
     const int k = e >> 4, c = e & 15;
     cp_async16(Wv + k * LDK + c * 8, W_UKV + (size_t)k * ldw + (size_t)h * 256 + 128 + c * 8);
   }
-  // merge weights per (sequence, chunk): w_s = 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c)
-  if (threadIdx.x < CMB_SEQ) {
-    const int r = threadIdx.x, i = i0 + r;
-    int ns = 0;
-    if (i < n_seq) {
-      ns = min(NS, (offs[i + 1] - offs[i] + CHUNK - 1) / CHUNK);
-      float M = -INFINITY;
-      for (int s = 0; s < ns; ++s) M = fmaxf(M, part_ml[(((size_t)i * NS + s) * HEADS + h) * 2]);
-      float Ls = 0.f;
-      for (int s = 0; s < ns; ++s) {
-        const size_t k = (((size_t)i * NS + s) * HEADS + h) * 2;
-        const float w = ex2((part_ml[k] - M) * scale_log2);
-        wsc[r * NS + s] = w;
-        Ls += part_ml[k + 1] * w;
-      }
-      const float inv = 1.f / Ls;
-      for (int s = 0; s < ns; ++s) wsc[r * NS + s] *= inv;
-    }
-    nsv[r] = ns;
-  }
-  __syncthreads();
-  // merged, normalised latent u[i][:] in bf16: each thread owns 16 groups of
-  // four latents (rows r = tid/128 + 2k); the chunk loop is outermost so the
-  // 16 loads of one chunk are independent and in flight together.
-  constexpr int PER = CMB_SEQ * (LAT / 4) / 256;
-  float4 u[PER];
-  int maxns = 0;
-#pragma unroll
-  for (int k = 0; k < PER; ++k) { u[k] = make_float4(0.f, 0.f, 0.f, 0.f); maxns = max(maxns, nsv[(threadIdx.x + 256 * k) / (LAT / 4)]); }
-  for (int s = 0; s < maxns; ++s) {
-#pragma unroll
-    for (int k = 0; k < PER; ++k) {
-      const int e = threadIdx.x + 256 * k, r = e / (LAT / 4), l = (e % (LAT / 4)) * 4, i = i0 + r;
-      if (s < nsv[r]) {
-        const float w = wsc[r * NS + s];
-        const float4 v = *reinterpret_cast<const float4*>(part_u + (((size_t)i * NS + s) * HEADS + h) * LAT + l);
-        u[k].x = fmaf(v.x, w, u[k].x); u[k].y = fmaf(v.y, w, u[k].y);
-        u[k].z = fmaf(v.z, w, u[k].z); u[k].w = fmaf(v.w, w, u[k].w);
-      }
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int e = threadIdx.x + 256 * k, r = e / (LAT / 4), l = (e % (LAT / 4)) * 4;
-    __nv_bfloat162* d = reinterpret_cast<__nv_bfloat162*>(U + r * LDU + l);
-    d[0] = __floats2bfloat162_rn(u[k].x, u[k].y);
-    d[1] = __floats2bfloat162_rn(u[k].z, u[k].w);
+  for (int e = threadIdx.x; e < PRJ_SEQ * (LAT / 8); e += blockDim.x) {
+    const int r = e / (LAT / 8), c = e % (LAT / 8), i = i0 + r;
+    if (i < n_seq) cp_async16(U + r * LDU + c * 8, u_in + ((size_t)i * HEADS + h) * LAT + c * 8);
+    else *reinterpret_cast<uint4*>(U + r * LDU + c * 8) = make_uint4(0u, 0u, 0u, 0u);
   }
   cp_async_wait_all();
   __syncthreads();
-  // O[i][h][:] = u W_UV,h  (M = 32 sequences, N = 128, K = 512)
-  float acc[2][2][4] = {};
+  float acc[4][2][4] = {};
 #pragma unroll 4
   for (int kk = 0; kk < LAT / 16; ++kk) {
     const int k0 = kk * 16;
@@ -463,7 +454,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int n_seq, int NS, const i
     for (int nt = 0; nt < 2; ++nt)
       ldsm_x2_trans(bf[nt][0], bf[nt][1], Wv + (k0 + (lane & 15)) * LDK + warp * 16 + nt * 8);
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
+    for (int mt = 0; mt < 4; ++mt) {
       const __nv_bfloat16* ar = U + (mt * 16 + gq) * LDU + k0 + 2 * t;
       const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDU), lds32(ar + 8), lds32(ar + 8 * LDU + 8)};
 #pragma unroll
@@ -471,7 +462,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int n_seq, int NS, const i
     }
   }
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -490,14 +481,14 @@ __global__ void __launch_bounds__(256) combine_kernel(int n_seq, int NS, const i
       }
 }
 
-inline size_t combine_smem(int NS) { return (size_t)LAT * LDK * 2 + (size_t)CMB_SEQ * LDU * 2 + (size_t)CMB_SEQ * NS * 4 + CMB_SEQ * 4; }
 
 inline int splits(int max_len) { return (max_len + CHUNK - 1) / CHUNK; }
 
 inline size_t workspace_bytes(int n, int max_len) {
   auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
   const size_t ns = splits(max_len);
-  return al((size_t)n * HEADS * WID * 2) + al((size_t)n * ns * HEADS * 2 * 4) + al((size_t)n * ns * HEADS * LAT * 4);
+  return al((size_t)n * HEADS * WID * 2) + al((size_t)n * ns * HEADS * 2 * 4) + al((size_t)n * ns * HEADS * LAT * 4) +
+         al((size_t)n * HEADS * LAT * 2);
 }
 
 }  // namespace tc_dec
