@@ -141,12 +141,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, SplitParams p) {
       for (int j = 0; ok && j < nt;) {
         bool progressed = false;
         if (next_qk < nt && next_qk <= j + 1 &&
-            mbar_try_wait(bar(CFULL + next_qk % NSTAGE), (next_qk / NSTAGE) & 1)) {
+            mbar_test(bar(CFULL + next_qk % NSTAGE), (next_qk / NSTAGE) & 1)) {
           tc_fence_after();
           issue_qk(next_qk++);
           progressed = true;
         }
-        if (next_qk > j && mbar_try_wait(bar(PFULL), j & 1)) {
+        if (next_qk > j && mbar_test(bar(PFULL), j & 1)) {
           tc_fence_after();
           const uint32_t cst = sbase + OFF_C + (j % NSTAGE) * STAGE;
 #pragma unroll
@@ -215,13 +215,16 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, SplitParams p) {
       tmem_ld32(tmem + lane_off + TM_S + (uint32_t)(j & 1) * 64u + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
       tmem_wait_ld();
       const int ws = window(j);
-      float mx = -INFINITY;
+      float pm[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
 #pragma unroll
       for (int k = 0; k < BT; ++k) {
         const int tok = ws + k;
         s[k] = (upper && tok >= j * BT && tok < len) ? s[k] : -INFINITY;
-        mx = fmaxf(mx, s[k]);
+        pm[k & 7] = fmaxf(pm[k & 7], s[k]);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       const bool need = upper && head_ok && mx > m_used + thr_add;     // first tile: m_used = -inf
       const float m_new = need ? mx : m_used;
       const float corr = need ? ex2((m_used - m_new) * c) : 1.f;       // 0 on the first tile
@@ -253,17 +256,19 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, SplitParams p) {
         // Rows of the 16 idle heads (48-63) get P = 0.
         const float neg = head_ok ? -m_used * c : 0.f;
         const uint32_t prow = sbase + OFF_P + (uint32_t)hr * 128u;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           float e[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             e[q] = head_ok ? ex2(fmaf(s[8 * cc + q], c, neg)) : 0.f;
-            lsum += e[q];
+            ps[q] += e[q];
           }
           st_shared_v4(prow + ((uint32_t)(cc ^ (hr & 7)) << 4), pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
                        pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
         }
+        lsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       }
       fence_proxy_async_smem();
       tc_fence_before();
