@@ -113,7 +113,7 @@ static bool is_k3_decode_geometry(const gmla_geom* g) {
 
 static size_t decode_ws_bytes(const gmla_geom* g, gmla_dtype dtype, int n, int max_len) {
   size_t b = simt::decode_workspace(g->H, g->kv_lora, g->d_s, n, max_len);
-  if (dtype == GMLA_BF16 && is_k3_decode_geometry(g)) b = std::max(b, tc_dec::workspace_bytes(n, max_len));
+  if (dtype == GMLA_BF16 && is_k3_decode_geometry(g)) b = std::max(b, tc_dec::workspace_bytes(n));
   return b;
 }
 
@@ -132,31 +132,40 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
                                       (int)tc_dec::ABS_SMEM);
   });
   if (attr_err != cudaSuccess) return cuda_status(attr_err);
-  const int NS = tc_dec::splits(max_len);
+  // One split CTA per SM (at most G_CAP), never more CTAs than tiles can exist.
+  int dev = 0, sms = 0;
+  GMLA_TRY(cuda_status(cudaGetDevice(&dev)));
+  GMLA_TRY(cuda_status(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)));
+  const long long max_tiles = (long long)n * ((max_len + tc_dec::BT - 1) / tc_dec::BT);
+  const int G = (int)std::max<long long>(1, std::min<long long>(std::min(sms, tc_dec::G_CAP), max_tiles));
   using bf = __nv_bfloat16;
   auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
+  const size_t np = (size_t)tc_dec::G_CAP + n;
   char* p = static_cast<char*>(ws);
   bf* q_abs = reinterpret_cast<bf*>(p);
   p += al((size_t)n * tc_dec::HEADS * tc_dec::WID * 2);
+  int* plan = reinterpret_cast<int*>(p);
+  p += al(((size_t)n + 1 + tc_dec::G_CAP) * 4);
   float* part_ml = reinterpret_cast<float*>(p);
-  p += al((size_t)n * NS * tc_dec::HEADS * 2 * 4);
+  p += al(np * tc_dec::HEADS * 2 * 4);
   float* part_u = reinterpret_cast<float*>(p);
-  p += al((size_t)n * NS * tc_dec::HEADS * tc_dec::LAT * 4);
+  p += al(np * tc_dec::HEADS * tc_dec::LAT * 4);
   bf* u_merged = reinterpret_cast<bf*>(p);
-  CUtensorMap mC;
+  CUtensorMap mC, mQ;
   // Rows of the cache map: every row a tile reads lies inside some sequence
-  // (the last tile of a chunk is shifted back to end at the chunk's end), so
+  // (the last tile of a sequence is shifted back to end at its end), so
   // n * max_len bounds the coordinates that occur; rows before 0 read as zero.
   const uint64_t rows = std::min<uint64_t>((uint64_t)n * (uint64_t)max_len, 0x7fffffffull);
   GMLA_TRY(make_map_2d(&mC, cache, tc_dec::WID, rows, tc_dec::BT));
+  GMLA_TRY(make_map_2d(&mQ, q_abs, tc_dec::WID, (uint64_t)n * tc_dec::HEADS, tc_dec::HEADS));
   tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256, tc_dec::ABS_SMEM, st>>>(
-      n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs);
+      n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs, offs, G, plan);
   tc_dec::SplitParams sp;
-  sp.n_seq = n; sp.NS = NS; sp.offs = offs; sp.q_abs = q_abs;
+  sp.n_seq = n; sp.G = G; sp.offs = offs; sp.plan = plan;
   sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   sp.part_ml = part_ml; sp.part_u = part_u;
-  tc_dec::decode_split_kernel<<<dim3(2, NS, n), 192, tc_dec::SMEM_BYTES, st>>>(mC, sp);
-  tc_dec::merge_kernel<<<(n * tc_dec::HEADS + 7) / 8, 256, 0, st>>>(n, NS, offs, sp.scale_log2, part_ml, part_u, u_merged);
+  tc_dec::decode_split_kernel<<<G, 192, tc_dec::SMEM_BYTES, st>>>(mC, mQ, sp);
+  tc_dec::merge_kernel<<<(n * tc_dec::HEADS + 7) / 8, 256, 0, st>>>(n, G, plan, sp.scale_log2, part_ml, part_u, u_merged);
   tc_dec::project_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::PRJ_SEQ - 1) / tc_dec::PRJ_SEQ), 256, tc_dec::PRJ_SMEM, st>>>(
       n, u_merged, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate), static_cast<bf*>(O));
   note_launches(4);

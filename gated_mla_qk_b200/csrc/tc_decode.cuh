@@ -8,21 +8,31 @@
 //   q~_h = [q^C_h W_UK,h^T | q^S_h]                          (absorb kernel)
 //   s_j  = q~_h . cache_j / sqrt(192), p = softmax_j(s)
 //   u_h  = sum_j p_j cache_j[0:512]                          (split kernel)
-//   o_h  = (u_h / l) W_UV,h  (* sigmoid(g))                  (combine kernel)
+//   o_h  = (u_h / l) W_UV,h  (* sigmoid(g))                  (merge + project kernels)
 //
-// Split kernel: one CTA per (sequence, 1024-token chunk, half of the heads).
-// Heads sit on the MMA's M side (48 heads as an M = 64 tile, half the TMEM
-// lanes), tokens on N:
-//   S [48 heads x 64 tokens] = q~ (A, resident in TMEM) x cache_tile^T (B, K-major)
-//   U [48 heads x 512]      += P (A, smem) x cache_tile (B, MN-major)
-// so the 64-token tile of the latent cache, streamed through three 72 KB TMA
-// stages, is the only operand read from shared memory by the score product,
-// and the same 128B-swizzled tile serves both products.  q~ and S live in the
-// upper half of each TMEM sub-partition, U in the lower half.  Softmax is per
-// row (one head per thread) with a lazily updated reference max; a row of U
-// is rescaled only when its max grows by more than 2^8, and only while no
-// product of this CTA is in flight.  Each CTA writes its partial (reference
-// max, sum, U) in fp32; the combine kernel merges the chunks and applies W_UV.
+// Split kernel: a persistent grid of one CTA per SM.  The 64-token tiles of
+// all sequences, laid end to end, are cut into equal ranges, one per CTA, so
+// every SM streams the same number of cache bytes whatever the length mix; a
+// range may end in the middle of one sequence and start in the middle of
+// another.  Each (CTA, sequence) piece of a range writes one partial (the
+// reference max, sum and U of every head) that the merge kernel combines.
+//
+// Per 64-token tile, both products run on the tensor core at M = 128:
+//   S   [96(+32) heads x 64 tokens] = q~ (A, smem, K-major) x tile^T (B, K-major)
+//   U^T [512 latent x 96 heads]    += tile^T (A, smem, MN-major) x P^T (B, K-major)
+// All 96 heads share one read of the tile.  Heads sit on M for the score
+// product (one softmax row per thread), and the latent sits on M for the
+// value product, so U^T takes 4 x 96 TMEM columns beside the two 64-column
+// S buffers.  q~ (108 KB) stays in shared memory for the whole sequence; the
+// tile streams through a ring of six 16 KB slots (a 128-wide latent pair
+// each) and one 8 KB slot for the 64 shared-key dims.  The score product of
+// tile t+1 starts on the slots that are free while the softmax of tile t
+// runs; the value product of tile t then frees the pair slots one by one for
+// the rest of tile t+1.
+// Softmax: base-2 exponentials against a lazily updated reference max per
+// head; U^T's column of a head is rescaled only when the head's max grows by
+// more than 2^8 (all four softmax warps take part, since a head's column
+// spans every TMEM lane).
 #pragma once
 
 #include "sm100.cuh"
@@ -32,60 +42,95 @@ namespace tc_dec {
 
 using namespace sm100;
 
-constexpr int HEADS = 96, HH = 48;        // heads, heads per CTA (an M = 64 tile with 16 idle rows)
-constexpr int BT = 64;                     // tokens per tile (N of the score product)
-constexpr int CHUNK = 1024;                // tokens per split (work item)
-constexpr int LAT = 512, WID = 576, NSUB = 9, NSTAGE = 3;
-constexpr uint32_t CSUB = BT * 128;        // one [64 tokens x 64] bf16 sub-tile of the cache (8 KB)
-constexpr uint32_t STAGE = NSUB * CSUB;    // 72 KB
-constexpr uint32_t OFF_C = 0;
-constexpr uint32_t OFF_P = OFF_C + NSTAGE * STAGE;          // P [64 head rows x 128 B]
-constexpr uint32_t OFF_BAR = OFF_P + CSUB;
+constexpr int HEADS = 96, BT = 64, LAT = 512, WID = 576;
+constexpr int NLP = 6;                     // latent-pair ring slots
+constexpr int G_CAP = 256;                 // most split CTAs (one per SM)
+constexpr uint32_t CSUB = BT * 128;        // [64 tokens x 64 dims] bf16, 8 KB
+constexpr uint32_t PAIR = 2 * CSUB;        // one 128-wide latent pair, 16 KB
+constexpr uint32_t QCH = HEADS * 128;      // [96 heads x 64 dims] bf16, 12 KB
+constexpr uint32_t OFF_Q = 0;              // q~: 9 chunks of 64 dims
+constexpr uint32_t OFF_P = OFF_Q + 9 * QCH;                 // P^T [96 heads x 64 tokens]
+constexpr uint32_t OFF_LAT = OFF_P + QCH;
+constexpr uint32_t OFF_ROPE = OFF_LAT + NLP * PAIR;
+constexpr uint32_t OFF_CORR = OFF_ROPE + CSUB;              // 96 rescale factors
+constexpr uint32_t OFF_BAR = OFF_CORR + 512;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-// TMEM columns.  Upper lanes (0-15 of each sub-partition): q~ as the A operand
-// (576 bf16 = 288 columns) and two S buffers; lower lanes (16-31): U.
-constexpr uint32_t TM_Q = 0, TM_S = 288, TM_U = 0;
-constexpr uint32_t LANE_LO = 16u << 16;   // lane offset of the lower half
+constexpr uint32_t TM_S = 0, TM_U = 128;   // TMEM columns: S buffers 2 x 64, U^T 4 x 96
+// The score product reads 128 rows of each q~ chunk: rows 96-127 fall on the
+// next chunk (or on P^T for the last one), and the S rows they give are never
+// read.
 
-enum Bar { CFULL = 0, CEMPTY = CFULL + NSTAGE, SFULL = CEMPTY + NSTAGE, PFULL = SFULL + 2, PVDONE = PFULL + 1,
-           QREADY = PVDONE + 1, DRAIN = QREADY + 1, NBAR = DRAIN + 1 };
+enum Bar { QFULL = 0, QEMPTY, LFULL, LEMPTY = LFULL + NLP, RFULL = LEMPTY + NLP, REMPTY, SFULL,
+           PFULL = SFULL + 2, SEGDONE, UFREE, DRAIN, NBAR };
 
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kPrefetchAhead = 2;          // tiles brought into L2 beyond the stages
+constexpr int kPrefetchAhead = 3;          // tiles brought into L2 ahead of their ring loads
 
 struct SplitParams {
-  int n_seq, NS;
+  int n_seq, G;
   const int* offs;                 // [n_seq + 1]
-  const __nv_bfloat16* q_abs;      // [n][96][576]
+  const int* plan;                 // [n_seq + 1] tile prefix, then [G] first sequence of each CTA
   float scale_log2;                // log2(e) / sqrt(192)
-  float* part_ml;                  // [n][NS][96][2]: reference max (raw logit units), sum
-  float* part_u;                   // [n][NS][96][512]
+  float* part_ml;                  // [G + n_seq][96][2]: reference max (raw logit units), sum
+  float* part_u;                   // [G + n_seq][96][512]
 };
 
+// Walks the tiles of a CTA's range: sequence i, tile k of it.  The tile's
+// 64-row window ends at the sequence's end when the tile is the last one, so
+// no row past the sequence (or the cache) is read; rows before the sequence
+// are masked (and rows before the cache read as zero).
+struct TileCursor {
+  const int* offs;
+  int n, i, k, nti, L, start;
+  __device__ void load(int seq) {
+    i = seq;
+    if (seq < n) { start = offs[seq]; L = offs[seq + 1] - start; nti = (L + BT - 1) / BT; }
+  }
+  __device__ void next() {
+    if (++k == nti) { k = 0; load(i + 1); }
+  }
+  __device__ int wrel() const { return min(k * BT, L - BT); }
+  __device__ int row() const { return start + wrel(); }
+  __device__ bool last_of_seq() const { return k == nti - 1; }
+};
+
+__device__ __forceinline__ void cta_range(const int* plan, int n, int G, int c, int& nt, int& i0, int& k0) {
+  const long long N = plan[n];
+  const long long t0 = (long long)c * N / G, t1 = (long long)(c + 1) * N / G;
+  nt = (int)(t1 - t0);
+  i0 = nt > 0 ? plan[n + 1 + c] : 0;
+  k0 = nt > 0 ? (int)(t0 - plan[i0]) : 0;
+}
+
 __global__ void __launch_bounds__(192, 1)
-decode_split_kernel(const __grid_constant__ CUtensorMap tmC, SplitParams p) {
+decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmQ, SplitParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  float* corr_sm = reinterpret_cast<float*>(smem_raw + (sbase - sraw) + OFF_CORR);
   volatile int* abort = &abort_flag;
   auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
-
-  const int hh = blockIdx.x, split = blockIdx.y, seq = blockIdx.z;
-  const int beg = p.offs[seq], L = p.offs[seq + 1] - beg;
-  const int t0 = split * CHUNK;
-  if (t0 >= L) return;                                   // whole CTA: no work in this chunk
-  const int len = min(CHUNK, L - t0);
-  const int nt = (len + BT - 1) / BT;
-  const int row0 = beg + t0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+
+  int nt, i0, k0;
+  cta_range(p.plan, p.n_seq, p.G, cta, nt, i0, k0);
+  if (nt == 0) return;                                   // whole CTA: empty range
+  auto cursor = [&]() {
+    TileCursor cur;
+    cur.offs = p.offs; cur.n = p.n_seq; cur.k = k0;
+    cur.load(i0);
+    return cur;
+  };
 
   if (threadIdx.x == 0) abort_flag = device_error_pending() ? 1 : 0;
   __syncthreads();
   if (abort_flag) return;
+  __syncthreads();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == PFULL || i == QREADY) ? 128 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == PFULL || i == UFREE) ? 128 : 1);
     fence_mbar_init();
   }
   if (warp == 5) { tmem_alloc(smem_u32(&tmem_slot), 512); tmem_relinquish(); }
@@ -94,205 +139,269 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, SplitParams p) {
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
-  // Rows [ws, ws + 64) of tile j relative to row0; the last tile is shifted
-  // back so that no row past the chunk's end is read.
-  auto window = [&](int j) { return min(j * BT, len - BT); };
-
   if (warp == 4) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmC);
-      auto prefetch = [&](int j) {
-        if (j < nt)
-          for (int k = 0; k < NSUB; ++k) tma_prefetch_l2_2d(&tmC, 64 * k, row0 + window(j));
+      tma_prefetch_desc(&tmC); tma_prefetch_desc(&tmQ);
+      TileCursor cur = cursor(), pf = cursor();
+      int pf_t = 0;
+      auto prefetch_upto = [&](int upto) {
+        for (; pf_t < upto && pf_t < nt; ++pf_t) {
+          for (int x = 0; x < 9; ++x) tma_prefetch_l2_2d(&tmC, 64 * x, pf.row());
+          pf.next();
+        }
       };
-      for (int j = NSTAGE; j < NSTAGE + kPrefetchAhead; ++j) prefetch(j);
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
-        const uint32_t st = j % NSTAGE, ph = (j / NSTAGE) & 1;
-        if (!mbar_wait(bar(CEMPTY + st), ph ^ 1u, abort)) break;
-        prefetch(j + NSTAGE + kPrefetchAhead);
-        mbar_arrive_expect_tx(bar(CFULL + st), STAGE);
-        const int r = row0 + window(j);
-        for (int k = 0; k < NSUB; ++k)
-          tma_load_2d(sbase + OFF_C + st * STAGE + k * CSUB, &tmC, bar(CFULL + st), 64 * k, r);
-        ++issued;
+      int seg = 0, lat_issued = 0, rope_issued = 0;
+      bool ok = true;
+      for (int t = 0; ok && t < nt; ++t) {
+        if (t == 0 || cur.k == 0) {
+          if (t > 0) {
+            ++seg;
+            if (!mbar_wait(bar(QEMPTY), (uint32_t)(seg - 1) & 1u, abort)) { ok = false; break; }
+          }
+          mbar_arrive_expect_tx(bar(QFULL), 9 * QCH);
+          for (int c = 0; c < 9; ++c) tma_load_2d(sbase + OFF_Q + c * QCH, &tmQ, bar(QFULL), 64 * c, cur.i * HEADS);
+        }
+        prefetch_upto(t + 1 + kPrefetchAhead);
+        const int row = cur.row();
+        // Ring order = the order the MMA thread consumes: pairs 0, 1, the
+        // shared-key dims, pairs 2, 3.
+        for (int q = 0; q < 5 && ok; ++q) {
+          if (q == 2) {
+            if (!mbar_wait(bar(REMPTY), ((uint32_t)t & 1u) ^ 1u, abort)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar(RFULL), CSUB);
+            tma_load_2d(sbase + OFF_ROPE, &tmC, bar(RFULL), LAT, row);
+            ++rope_issued;
+          } else {
+            const int pr = q < 2 ? q : q - 1;
+            const int u = 4 * t + pr;
+            const uint32_t slot = (uint32_t)(u % NLP);
+            if (!mbar_wait(bar(LEMPTY + slot), ((uint32_t)(u / NLP) & 1u) ^ 1u, abort)) { ok = false; break; }
+            const uint32_t dst = sbase + OFF_LAT + slot * PAIR;
+            mbar_arrive_expect_tx(bar(LFULL + slot), PAIR);
+            tma_load_2d(dst, &tmC, bar(LFULL + slot), 128 * pr, row);
+            tma_load_2d(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row);
+            lat_issued = u + 1;
+          }
+        }
+        cur.next();
       }
-      for (int j = (issued > NSTAGE ? issued - NSTAGE : 0); j < issued; ++j)
-        mbar_wait_drain(bar(CFULL + j % NSTAGE), (j / NSTAGE) & 1);
+      // Never leave with copies in flight into this CTA's shared memory.
+      mbar_wait_drain(bar(QFULL), (uint32_t)seg & 1u);
+      if (rope_issued > 0) mbar_wait_drain(bar(RFULL), (uint32_t)(rope_issued - 1) & 1u);
+      for (int u = (lat_issued > NLP ? lat_issued - NLP : 0); u < lat_issued; ++u)
+        mbar_wait_drain(bar(LFULL + u % NLP), (uint32_t)(u / NLP) & 1u);
     }
   } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idQK = idesc_bf16_f32(64, BT, false, false);    // q~ (TMEM) x cache tile (K-major)
-      constexpr uint32_t idPV = idesc_bf16_f32(64, 256, false, true);    // P (K-major) x cache tile (MN-major)
-      auto issue_qk = [&](int j) {
-        const uint32_t cst = sbase + OFF_C + (j % NSTAGE) * STAGE;
-        const uint32_t d = tmem + TM_S + (uint32_t)(j & 1) * 64u;
-#pragma unroll
-        for (int i = 0; i < 4 * NSUB; ++i)
-          mma_ts(d, tmem + TM_Q + 8u * i, sdesc_sw128(cst + (i >> 2) * CSUB + (i & 3) * 32, 16, 1024), idQK, i != 0);
-        mma_commit(bar(SFULL + (j & 1)));
+      constexpr uint32_t idQK = idesc_bf16_f32(128, BT, false, false);      // q~ (K-major) x tile (K-major)
+      constexpr uint32_t idPV = idesc_bf16_f32(128, HEADS, true, false);    // tile^T (MN-major) x P^T (K-major)
+      bool ok = true;
+      auto wait_ok = [&](int b, uint32_t ph) {
+        ok = ok && mbar_wait(bar(b), ph, abort);
+        if (ok) tc_fence_after();
+        return ok;
       };
-      // Event loop: issue the score product of a tile as soon as its data has
-      // landed (and its S buffer is free), and the P.V product of tile j as
-      // soon as P is written, in whichever order they become ready.
-      bool ok = mbar_wait(bar(QREADY), 0, abort);
-      int next_qk = 0;
-      uint64_t t_start = 0;
-      for (int j = 0; ok && j < nt;) {
-        bool progressed = false;
-        if (next_qk < nt && next_qk <= j + 1 &&
-            mbar_test(bar(CFULL + next_qk % NSTAGE), (next_qk / NSTAGE) & 1)) {
-          tc_fence_after();
-          issue_qk(next_qk++);
-          progressed = true;
-        }
-        if (next_qk > j && mbar_test(bar(PFULL), j & 1)) {
-          tc_fence_after();
-          const uint32_t cst = sbase + OFF_C + (j % NSTAGE) * STAGE;
+      // Score product of tile t: q~ chunks 2pr, 2pr+1 against latent pair pr.
+      auto qk_pair = [&](int t, int pr, bool first) {
+        const int u = 4 * t + pr;
+        const uint32_t slot = (uint32_t)(u % NLP);
+        if (!wait_ok(LFULL + slot, (uint32_t)(u / NLP) & 1u)) return;
+        const uint32_t sb = sbase + OFF_LAT + slot * PAIR;
+        const uint32_t d = tmem + TM_S + (uint32_t)(t & 1) * BT;
 #pragma unroll
-          for (int kk = 0; kk < BT / 16; ++kk)
+        for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-            for (int nh = 0; nh < 2; ++nh)
-              mma_ss(tmem + LANE_LO + TM_U + 256u * nh, sdesc_sw128(sbase + OFF_P + kk * 32, 16, 1024),
-                     sdesc_sw128(cst + (4 * nh) * CSUB + kk * 2048, CSUB, 1024), idPV, (j > 0 || kk > 0));
-          mma_commit(bar(PVDONE));
-          mma_commit(bar(CEMPTY + j % NSTAGE));
-          ++j;
-          progressed = true;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(d, sdesc_sw128(sbase + OFF_Q + (uint32_t)(2 * pr + hf) * QCH + kk * 32u, 16, 1024),
+                   sdesc_sw128(sb + hf * CSUB + kk * 32u, 16, 1024), idQK, !(first && hf == 0 && kk == 0));
+      };
+      auto qk_rope = [&](int t) {
+        if (!wait_ok(RFULL, (uint32_t)t & 1u)) return;
+        const uint32_t d = tmem + TM_S + (uint32_t)(t & 1) * BT;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(d, sdesc_sw128(sbase + OFF_Q + 8u * QCH + kk * 32u, 16, 1024),
+                 sdesc_sw128(sbase + OFF_ROPE + kk * 32u, 16, 1024), idQK, true);
+        mma_commit(bar(REMPTY));
+      };
+      // Value product of tile t, one 128-row latent block per pair; each
+      // pair slot is released as soon as its block is issued.
+      auto pv = [&](int t, bool fresh) {
+#pragma unroll 1
+        for (int b = 0; b < 4; ++b) {
+          const int u = 4 * t + b;
+          const uint32_t slot = (uint32_t)(u % NLP);
+          const uint32_t sb = sbase + OFF_LAT + slot * PAIR;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + TM_U + (uint32_t)b * HEADS, sdesc_sw128(sb + kk * 2048u, CSUB, 1024),
+                   sdesc_sw128(sbase + OFF_P + kk * 32u, 16, 1024), idPV, !(fresh && kk == 0));
+          mma_commit(bar(LEMPTY + slot));
         }
-        if (progressed) { t_start = 0; continue; }
-        if (*abort || device_error_pending()) { *abort = 1; ok = false; break; }
-        const uint64_t now = globaltimer_ns();
-        if (t_start == 0) t_start = now;
-        else if (now - t_start > kWaitLimitNs) { raise_device_error(GMLA_ETIMEOUT); *abort = 1; ok = false; }
+      };
+      TileCursor cur = cursor(), nxt = cursor();
+      nxt.next();
+      int seg = 0;
+      // Score product of the first tile.
+      if (wait_ok(QFULL, 0)) {
+        qk_pair(0, 0, true); qk_pair(0, 1, false); qk_rope(0); qk_pair(0, 2, false); qk_pair(0, 3, false);
+        mma_commit(bar(SFULL));
+        if (nt == 1 || cur.last_of_seq()) mma_commit(bar(QEMPTY));
       }
+      for (int t = 0; ok && t < nt; ++t) {
+        const bool first = (t == 0) || cur.k == 0;
+        const bool last = (t == nt - 1) || cur.last_of_seq();
+        const bool pre = (t + 1 < nt) && !last;           // tile t+1 continues this sequence
+        if (pre) { qk_pair(t + 1, 0, true); qk_pair(t + 1, 1, false); qk_rope(t + 1); }
+        if (!wait_ok(PFULL, (uint32_t)t & 1u)) break;
+        if (first && seg > 0 && !wait_ok(UFREE, (uint32_t)(seg - 1) & 1u)) break;
+        pv(t, first);
+        if (last) mma_commit(bar(SEGDONE));
+        if (t + 1 < nt) {
+          if (pre) {
+            qk_pair(t + 1, 2, false); qk_pair(t + 1, 3, false);
+          } else {
+            ++seg;
+            if (!wait_ok(QFULL, (uint32_t)seg & 1u)) break;
+            qk_pair(t + 1, 0, true); qk_pair(t + 1, 1, false); qk_rope(t + 1); qk_pair(t + 1, 2, false);
+            qk_pair(t + 1, 3, false);
+          }
+          if (!ok) break;
+          mma_commit(bar(SFULL + ((t + 1) & 1)));
+          if (t + 2 == nt || nxt.last_of_seq()) mma_commit(bar(QEMPTY));
+        }
+        cur.next();
+        nxt.next();
+      }
+      // Drain every MMA this thread issued before TMEM is released.
       mma_commit(bar(DRAIN));
       mbar_wait_drain(bar(DRAIN), 0);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-3)
-    // Lanes 0-15 of warp w own head rows 16w + lane (upper TMEM lanes: q~, S);
-    // lanes 16-31 hold the U rows of the same heads (lower TMEM lanes).
+    // ------------------------------------------------------------ softmax + partials (warps 0-3)
+    // Thread x owns head row x of S (x < 96) and latent row x of each U^T block.
+    const int x = threadIdx.x;
+    const bool head = x < HEADS;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float c = p.scale_log2;
     const float thr_add = kRescaleLog2 / c;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const bool upper = lane < 16;
-    const int hr = warp * 16 + (lane & 15);              // head row inside the CTA (valid if < 48)
-    const bool head_ok = hr < HH;
-    // Load q~ into the upper TMEM lanes (the lower lanes write zeros into the
-    // U columns, which the first P.V product overwrites).
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + ((size_t)seq * HEADS + hh * HH + (head_ok ? hr : 0)) * WID);
-#pragma unroll 1
-      for (int cch = 0; cch < 9; ++cch) {
-        float v[32];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 x = make_uint4(0u, 0u, 0u, 0u);
-          if (upper && head_ok) x = src[cch * 8 + q];
-          v[4 * q + 0] = __uint_as_float(x.x); v[4 * q + 1] = __uint_as_float(x.y);
-          v[4 * q + 2] = __uint_as_float(x.z); v[4 * q + 3] = __uint_as_float(x.w);
-        }
-        tmem_st32(tmem + lane_off + TM_Q + 32u * cch, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(QREADY));
-    }
-    float m_used = -INFINITY, lsum = 0.f;
+    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    auto wait_warp = [&](int i, uint32_t ph) {
-      const bool w = ok && mbar_wait(bar(i), ph, abort);
-      ok = __all_sync(0xffffffffu, w) != 0;
-      return ok;
-    };
-    for (int j = 0; j < nt && ok; ++j) {
-      if (!wait_warp(SFULL + (j & 1), (j >> 1) & 1)) break;
-      tc_fence_after();
+    int seg = 0;
+    TileCursor cur = cursor();
+    // The loop runs the same named barriers in every thread whatever
+    // happens, so a failed wait can never strand a warp in a barrier.
+    for (int t = 0; t < nt; ++t) {
+      const bool first = (t == 0) || cur.k == 0;
+      const bool last = (t == nt - 1) || cur.last_of_seq();
+      if (ok) ok = mbar_wait(bar(SFULL + (t & 1)), (uint32_t)(t >> 1) & 1u, abort);
+      ok = !bar_red_or(1, 128, !ok);
       float s[BT];
-      tmem_ld32(tmem + lane_off + TM_S + (uint32_t)(j & 1) * 64u, *reinterpret_cast<float(*)[32]>(&s[0]));
-      tmem_ld32(tmem + lane_off + TM_S + (uint32_t)(j & 1) * 64u + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
-      tmem_wait_ld();
-      const int ws = window(j);
-      float pm[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < BT; ++k) {
-        const int tok = ws + k;
-        s[k] = (upper && tok >= j * BT && tok < len) ? s[k] : -INFINITY;
-        pm[k & 7] = fmaxf(pm[k & 7], s[k]);
-      }
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      const bool need = upper && head_ok && mx > m_used + thr_add;     // first tile: m_used = -inf
-      const float m_new = need ? mx : m_used;
-      const float corr = need ? ex2((m_used - m_new) * c) : 1.f;       // 0 on the first tile
-      // P buffer and U: the previous product must have finished.
-      if (j > 0 && !wait_warp(PVDONE, (j - 1) & 1)) break;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // Rare: rescale this warp's U rows.  No product of this CTA is in
-        // flight once the score product of tile j+1 (if issued) is done,
-        // because P.V of tile j waits for this warp's arrival below.
-        if (j + 1 < nt && !wait_warp(SFULL + ((j + 1) & 1), ((j + 1) >> 1) & 1)) break;
+      bool need = false;
+      float corr = 1.f, m_new = m_used;
+      if (ok) {
         tc_fence_after();
-        const float f = __shfl_sync(0xffffffffu, corr, lane & 15);   // lower lane takes its head's factor
-#pragma unroll 1
-        for (int cch = 0; cch < LAT / 32; ++cch) {
-          float u[32];
-          tmem_ld32(tmem + lane_off + TM_U + 32u * cch, u);
-          tmem_wait_ld();
-          if (!upper) {
+        const uint32_t ts = tmem + lane_off + TM_S + (uint32_t)(t & 1) * BT;
+        tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_ld32(ts + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[32]));
+        if (head) {
+          const int w = cur.wrel();
+          const int lo = cur.k * BT - w, hi = cur.L - w;   // valid columns [lo, hi)
+          float pm[8];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] *= f;
+          for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < BT; ++e) {
+            s[e] = (e >= lo && e < hi) ? s[e] : -INFINITY;
+            pm[e & 7] = fmaxf(pm[e & 7], s[e]);
           }
-          tmem_st32(tmem + lane_off + TM_U + 32u * cch, u);
+          const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+          need = mx > m_used + thr_add;                     // always on a piece's first tile
+          m_new = need ? mx : m_used;
+          corr = need ? ex2((m_used - m_new) * c) : 1.f;    // 0 on a piece's first tile
+          if (!first) corr_sm[x] = corr;
         }
+      }
+      const bool resc = bar_red_or(1, 128, ok && head && need && !first);
+      if (ok && resc) {
+        // Rare: scale the U^T columns of the heads whose max moved.  The
+        // value product of tile t-1 has finished (it was issued before the
+        // score product of tile t), and that of tile t waits for this
+        // thread's arrival below.
+#pragma unroll 1
+        for (int b = 0; b < 4; ++b)
+#pragma unroll 1
+          for (int cc = 0; cc < 3; ++cc) {
+            const uint32_t tu = tmem + lane_off + TM_U + (uint32_t)(b * HEADS + 32 * cc);
+            float u[32];
+            tmem_ld32(tu, u);
+            tmem_wait_ld_dep(u);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] *= corr_sm[32 * cc + e];
+            tmem_st32(tu, u);
+          }
         tmem_wait_st();
       }
-      lsum *= corr;
-      m_used = m_new;
-      if (upper) {
-        // Rows of the 16 idle heads (48-63) get P = 0.
-        const float neg = head_ok ? -m_used * c : 0.f;
-        const uint32_t prow = sbase + OFF_P + (uint32_t)hr * 128u;
+      if (ok && head) {
+        l *= corr;
+        m_used = m_new;
+        const float neg = -m_used * c;
+        const uint32_t prow = sbase + OFF_P + (uint32_t)x * 128u;
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
-          float e[8];
+          float e8[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            e[q] = head_ok ? ex2(fmaf(s[8 * cc + q], c, neg)) : 0.f;
-            ps[q] += e[q];
+            e8[q] = ex2(fmaf(s[8 * cc + q], c, neg));
+            ps[q] += e8[q];
           }
-          st_shared_v4(prow + ((uint32_t)(cc ^ (hr & 7)) << 4), pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
-                       pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
+          st_shared_v4(prow + ((uint32_t)(cc ^ (x & 7)) << 4), pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]),
+                       pack_bf16x2(e8[4], e8[5]), pack_bf16x2(e8[6], e8[7]));
         }
-        lsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(PFULL));
-    }
-    if (ok && wait_warp(PVDONE, (nt - 1) & 1)) {
-      tc_fence_after();
-      const size_t pbase = ((size_t)seq * p.NS + split) * HEADS + hh * HH;
-      if (upper && head_ok) {
-        p.part_ml[(pbase + hr) * 2 + 0] = m_used;
-        p.part_ml[(pbase + hr) * 2 + 1] = lsum;
+      if (ok) {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(PFULL));
       }
-      float* dst = p.part_u + (pbase + (head_ok ? hr : 0)) * LAT;
+      if (last) {
+        // End of this CTA's piece of sequence cur.i: write its partial.
+        bool w_ok = ok && mbar_wait(bar(SEGDONE), (uint32_t)seg & 1u, abort);
+        w_ok = __all_sync(0xffffffffu, w_ok) != 0;
+        ok = ok && w_ok;
+        if (ok) {
+          tc_fence_after();
+          const size_t id = (size_t)cta + (size_t)cur.i;
+          float* dst = p.part_u + id * HEADS * LAT + x;
 #pragma unroll 1
-      for (int cch = 0; cch < LAT / 32; ++cch) {
-        float u[32];
-        tmem_ld32(tmem + lane_off + TM_U + 32u * cch, u);
-        tmem_wait_ld();
-        if (!upper && head_ok) {
-          float4* d4 = reinterpret_cast<float4*>(dst + 32 * cch);
+          for (int b = 0; b < 4; ++b)
+#pragma unroll 1
+            for (int cc = 0; cc < 3; ++cc) {
+              float u[32];
+              tmem_ld32(tmem + lane_off + TM_U + (uint32_t)(b * HEADS + 32 * cc), u);
+              tmem_wait_ld_dep(u);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) d4[q] = make_float4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+              for (int e = 0; e < 32; ++e) dst[(size_t)(32 * cc + e) * LAT + 128 * b] = u[e];
+            }
+          if (head) {
+            p.part_ml[(id * HEADS + x) * 2 + 0] = m_used;
+            p.part_ml[(id * HEADS + x) * 2 + 1] = l;
+          }
+          tc_fence_before();
+          mbar_arrive(bar(UFREE));
         }
+        m_used = -INFINITY;
+        l = 0.f;
+        ++seg;
       }
+      cur.next();
     }
   }
   tc_fence_before();
@@ -324,6 +433,45 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t& r0, uint32_t& r1, const 
                : "=r"(r0), "=r"(r1) : "r"(smem_u32(p)));
 }
 
+// Work plan of the split kernel, built by one block of 256 threads:
+//   plan[0..n]        P_i = number of 64-token tiles of sequences 0..i-1
+//   plan[n+1+c]       the sequence holding tile floor(c P_n / G), c < G
+__device__ void build_plan(int n_seq, const int* __restrict__ offs, int G, int* __restrict__ plan) {
+  __shared__ int wsum[8];
+  __shared__ int carry;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) { carry = 0; plan[0] = 0; }
+  __syncthreads();
+  for (int base = 0; base < n_seq; base += 256) {
+    const int i = base + (int)threadIdx.x;
+    int x = i < n_seq ? (offs[i + 1] - offs[i] + BT - 1) / BT : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    int pre = carry;
+    for (int w = 0; w < warp; ++w) pre += wsum[w];
+    const int incl = pre + x;
+    if (i < n_seq) plan[i + 1] = incl;
+    __syncthreads();
+    if (threadIdx.x == 255) carry = incl;
+    __syncthreads();
+  }
+  const long long N = carry;
+  for (int c = threadIdx.x; c < G; c += 256) {
+    const long long t = (long long)c * N / G;
+    int lo = 0, hi = n_seq - 1;                  // largest i with P_i <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (plan[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    plan[n_seq + 1 + c] = lo;
+  }
+}
+
 constexpr int ABS_SEQ = 64;                    // sequences per absorb block
 constexpr int LDK = 136;                       // padded bf16 row of a 128-wide staged operand
 constexpr size_t ABS_SMEM = (size_t)(LAT + ABS_SEQ) * LDK * 2;
@@ -332,15 +480,18 @@ constexpr size_t ABS_SMEM = (size_t)(LAT + ABS_SEQ) * LDK * 2;
 // 8 warps.  W_UK,h (512 x 128, one 256-byte row segment per latent index)
 // and the block's q^C rows are staged in shared memory with 16-byte loads;
 // warp w computes latent columns [64w, 64w + 64).
+// Block (0, 0) also builds the split kernel's work plan.
 __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ W_UKV,
-                                                     __nv_bfloat16* __restrict__ q_abs) {
+                                                     __nv_bfloat16* __restrict__ q_abs, const int* __restrict__ offs,
+                                                     int G, int* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t asm_[];
   __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(asm_);      // [512][LDK]: W_UK,h[latent][k]
   __nv_bfloat16* As = Ws + LAT * LDK;                               // [64][LDK]: q^C[i][k]
   const int h = blockIdx.x, i0 = blockIdx.y * ABS_SEQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   constexpr size_t ldw = (size_t)HEADS * 256;
+  if (blockIdx.x == 0 && blockIdx.y == 0) build_plan(n_seq, offs, G, plan);
   for (int e = threadIdx.x; e < LAT * 16; e += blockDim.x) {
     const int n = e >> 4, c = e & 15;
     cp_async16(Ws + n * LDK + c * 8, W_UKV + (size_t)n * ldw + (size_t)h * 256 + c * 8);
@@ -385,23 +536,37 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
   }
 }
 
-// Merge the chunks of each (sequence, head): one warp per pair, 16 latents per
+// Merge the pieces of each (sequence, head): one warp per pair, 16 latents per
 // lane.  u = sum_s U_s 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c), in bf16.
-__global__ void __launch_bounds__(256) merge_kernel(int n_seq, int NS, const int* __restrict__ offs, float scale_log2,
+// The pieces of sequence i are those of the CTAs whose tile ranges meet the
+// sequence's tiles; CTA c's piece of sequence i is partial c + i.
+__global__ void __launch_bounds__(256) merge_kernel(int n_seq, int G, const int* __restrict__ plan, float scale_log2,
                                                     const float* __restrict__ part_ml, const float* __restrict__ part_u,
                                                     __nv_bfloat16* __restrict__ u_out) {
   const int pair = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (pair >= n_seq * HEADS) return;
   const int i = pair / HEADS, h = pair % HEADS;
-  const int ns = min(NS, (offs[i + 1] - offs[i] + CHUNK - 1) / CHUNK);
+  const long long N = plan[n_seq];
+  const long long t_lo = plan[i], t_hi = plan[i + 1] - 1;
+  __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(u_out + ((size_t)i * HEADS + h) * LAT);
+  if (t_hi < t_lo) {                         // no tiles (outside the API's contract): zeros
+#pragma unroll
+    for (int q = 0; q < 8; ++q) dst[lane + 32 * q] = __floats2bfloat162_rn(0.f, 0.f);
+    return;
+  }
+  // CTA holding tile t: the largest c with floor(c N / G) <= t.
+  const int c_lo = (int)(((t_lo + 1) * G - 1) / N), c_hi = (int)(((t_hi + 1) * G - 1) / N);
+  auto empty = [&](int cc) { return (long long)cc * N / G == (long long)(cc + 1) * N / G; };
   float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, part_ml[(((size_t)i * NS + s) * HEADS + h) * 2]);
+  for (int cc = c_lo; cc <= c_hi; ++cc)
+    if (!empty(cc)) M = fmaxf(M, part_ml[((size_t)(cc + i) * HEADS + h) * 2]);
   float4 acc[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
   float Ls = 0.f;
-  for (int s = 0; s < ns; ++s) {
-    const size_t k = ((size_t)i * NS + s) * HEADS + h;
+  for (int cc = c_lo; cc <= c_hi; ++cc) {
+    if (empty(cc)) continue;
+    const size_t k = (size_t)(cc + i) * HEADS + h;
     const float w = ex2((part_ml[2 * k] - M) * scale_log2);
     Ls += part_ml[2 * k + 1] * w;
     const float4* src = reinterpret_cast<const float4*>(part_u + k * LAT);
@@ -413,7 +578,6 @@ __global__ void __launch_bounds__(256) merge_kernel(int n_seq, int NS, const int
     }
   }
   const float inv = 1.f / Ls;
-  __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(u_out + ((size_t)i * HEADS + h) * LAT);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int l4 = lane + 32 * q;
@@ -487,13 +651,12 @@ __global__ void __launch_bounds__(256) project_kernel(int n_seq, const __nv_bflo
 }
 
 
-inline int splits(int max_len) { return (max_len + CHUNK - 1) / CHUNK; }
 
-inline size_t workspace_bytes(int n, int max_len) {
+inline size_t workspace_bytes(int n) {
   auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
-  const size_t ns = splits(max_len);
-  return al((size_t)n * HEADS * WID * 2) + al((size_t)n * ns * HEADS * 2 * 4) + al((size_t)n * ns * HEADS * LAT * 4) +
-         al((size_t)n * HEADS * LAT * 2);
+  const size_t np = (size_t)G_CAP + n;
+  return al((size_t)n * HEADS * WID * 2) + al(((size_t)n + 1 + G_CAP) * 4) + al(np * HEADS * 2 * 4) +
+         al(np * HEADS * LAT * 4) + al((size_t)n * HEADS * LAT * 2);
 }
 
 }  // namespace tc_dec

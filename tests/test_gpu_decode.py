@@ -60,3 +60,39 @@ def test_decode_64_sequences_1k_to_8k():
     got = _run(d, "bf16")
     want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
     assert rel_l2(got, want) <= TOL_BF16
+
+
+def _with_lengths(lens, seed, ramp=0.0, gate=False):
+    """decode_batch's q / W_UKV with the listed lengths and a fresh cache; with
+    ramp > 0 the cache rows of each sequence grow in magnitude along the
+    sequence, so the running max of every head moves often."""
+    d = synth.decode_batch(n_seq=len(lens), lo=1, hi=2, seed=seed, gate=gate)
+    rng = np.random.default_rng(seed + 1)
+    lens = np.array(lens)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    cache = rng.standard_normal((int(offs[-1]), 576)).astype(np.float32)
+    if ramp:
+        for i in range(len(lens)):
+            a, b = offs[i], offs[i + 1]
+            cache[a:b] *= (1.0 + ramp * np.arange(b - a) / max(1, b - a - 1))[:, None]
+    d.update(lens=lens, seq_offsets=offs, cache=synth.round_storage(cache, "bf16"))
+    return d
+
+
+def test_running_max_moves_often():
+    """Logits that grow along each sequence (by far more than the 2^8 rescale
+    threshold) exercise the rescale of the accumulated latent sums."""
+    d = _with_lengths((3000, 700, 64, 65), seed=41, ramp=6.0)
+    got = _run(d, "bf16")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
+    assert rel_l2(got, want) <= TOL_BF16
+
+
+def test_many_short_sequences():
+    """160 sequences of 1-200 tokens: work ranges start and end inside
+    sequences and most ranges hold several sequences."""
+    lens = np.random.default_rng(43).integers(1, 201, size=160)
+    d = _with_lengths(tuple(int(x) for x in lens), seed=44, gate=True)
+    got = _run(d, "bf16")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
+    assert rel_l2(got, want) <= TOL_BF16
