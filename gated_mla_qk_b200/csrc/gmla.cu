@@ -161,7 +161,7 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256, tc_dec::ABS_SMEM, st>>>(
       n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs, offs, G, plan);
   tc_dec::SplitParams sp;
-  sp.n_seq = n; sp.G = G; sp.offs = offs; sp.plan = plan;
+  sp.n_seq = n; sp.G = G; sp.offs = offs; sp.plan = plan; sp.cache = static_cast<const bf*>(cache);
   sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   sp.part_ml = part_ml; sp.part_u = part_u;
   tc_dec::decode_split_kernel<<<G, 192, tc_dec::SMEM_BYTES, st>>>(mC, mQ, sp);

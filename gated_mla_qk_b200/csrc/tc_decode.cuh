@@ -10,25 +10,26 @@
 //   u_h  = sum_j p_j cache_j[0:512]                          (split kernel)
 //   o_h  = (u_h / l) W_UV,h  (* sigmoid(g))                  (merge + project kernels)
 //
-// Split kernel: a persistent grid of one CTA per SM.  The 64-token tiles of
+// Split kernel: a persistent grid of one CTA per SM.  The 96-token tiles of
 // all sequences, laid end to end, are cut into equal ranges, one per CTA, so
 // every SM streams the same number of cache bytes whatever the length mix; a
 // range may end in the middle of one sequence and start in the middle of
 // another.  Each (CTA, sequence) piece of a range writes one partial (the
 // reference max, sum and U of every head) that the merge kernel combines.
 //
-// Per 64-token tile, both products run on the tensor core at M = 128:
-//   S   [96(+32) heads x 64 tokens] = q~ (A, smem, K-major) x tile^T (B, K-major)
+// Per 96-token tile, both products run on the tensor core at M = 128:
+//   S   [96(+32) heads x 96 tokens] = q~ (A, smem, K-major) x tile^T (B, K-major)
 //   U^T [512 latent x 96 heads]    += tile^T (A, smem, MN-major) x P^T (B, K-major)
-// All 96 heads share one read of the tile.  Heads sit on M for the score
-// product (one softmax row per thread), and the latent sits on M for the
-// value product, so U^T takes 4 x 96 TMEM columns beside the two 64-column
-// S buffers.  q~ (108 KB) stays in shared memory for the whole sequence; the
-// tile streams through a ring of six 16 KB slots (a 128-wide latent pair
-// each) and one 8 KB slot for the 64 shared-key dims.  The score product of
-// tile t+1 starts on the slots that are free while the softmax of tile t
-// runs; the value product of tile t then frees the pair slots one by one for
-// the rest of tile t+1.
+// All 96 heads share one read of the tile from HBM.  Heads sit on M for the
+// score product (one softmax row per thread), the latent sits on M for the
+// value product, so U^T takes 4 x 96 TMEM columns beside the 96-column S.
+// q~ (108 KB) stays in shared memory for the whole sequence.  The tile's
+// latent streams through a ring of three 24 KB slots twice: once, as 128-wide
+// latent pairs, for the score product, and once more (from L2, where the
+// first pass left it) for the value product after the softmax, so no slot is
+// held across the softmax and the ring stays short.  The 64 shared-key dims
+// have a slot of their own.  The score product of tile t+1 runs while the
+// softmax of tile t runs; S is released as soon as the softmax has loaded it.
 // Softmax: base-2 exponentials against a lazily updated reference max per
 // head; U^T's column of a head is rescaled only when the head's max grows by
 // more than 2^8 (all four softmax warps take part, since a head's column
@@ -42,33 +43,34 @@ namespace tc_dec {
 
 using namespace sm100;
 
-constexpr int HEADS = 96, BT = 64, LAT = 512, WID = 576;
-constexpr int NLP = 6;                     // latent-pair ring slots
+constexpr int HEADS = 96, BT = 96, LAT = 512, WID = 576;
+constexpr int NPS = 3;                     // latent-pair ring slots
 constexpr int G_CAP = 256;                 // most split CTAs (one per SM)
-constexpr uint32_t CSUB = BT * 128;        // [64 tokens x 64 dims] bf16, 8 KB
-constexpr uint32_t PAIR = 2 * CSUB;        // one 128-wide latent pair, 16 KB
+constexpr uint32_t CSUB = BT * 128;        // [96 tokens x 64 dims] bf16, 12 KB
+constexpr uint32_t PAIR = 2 * CSUB;        // one 128-wide latent pair, 24 KB
 constexpr uint32_t QCH = HEADS * 128;      // [96 heads x 64 dims] bf16, 12 KB
 constexpr uint32_t OFF_Q = 0;              // q~: 9 chunks of 64 dims
-constexpr uint32_t OFF_P = OFF_Q + 9 * QCH;                 // P^T [96 heads x 64 tokens]
-constexpr uint32_t OFF_LAT = OFF_P + QCH;
-constexpr uint32_t OFF_ROPE = OFF_LAT + NLP * PAIR;
+constexpr uint32_t OFF_P = OFF_Q + 9 * QCH;                 // P^T: two [96 heads x 64 tokens] sub-tiles
+constexpr uint32_t OFF_PAIR = OFF_P + 2 * QCH;
+constexpr uint32_t OFF_ROPE = OFF_PAIR + NPS * PAIR;
 constexpr uint32_t OFF_CORR = OFF_ROPE + CSUB;              // 96 rescale factors
 constexpr uint32_t OFF_BAR = OFF_CORR + 512;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t TM_S = 0, TM_U = 128;   // TMEM columns: S buffers 2 x 64, U^T 4 x 96
+constexpr uint32_t TM_S = 0, TM_U = 128;   // TMEM columns: S (96), U^T 4 x 96
 // The score product reads 128 rows of each q~ chunk: rows 96-127 fall on the
 // next chunk (or on P^T for the last one), and the S rows they give are never
 // read.
 
-enum Bar { QFULL = 0, QEMPTY, LFULL, LEMPTY = LFULL + NLP, RFULL = LEMPTY + NLP, REMPTY, SFULL,
-           PFULL = SFULL + 2, SEGDONE, UFREE, DRAIN, NBAR };
+enum Bar { QFULL = 0, QEMPTY, LFULL, LEMPTY = LFULL + NPS, RFULL = LEMPTY + NPS, REMPTY, SFULL, SFREE, PFULL,
+           PVDONE, UFREE, DRAIN, NBAR };
 
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kPrefetchAhead = 3;          // tiles brought into L2 ahead of their ring loads
+constexpr int kPrefetchAhead = 3;          // tiles brought into L2 ahead of their first ring load
 
 struct SplitParams {
   int n_seq, G;
   const int* offs;                 // [n_seq + 1]
+  const __nv_bfloat16* cache;      // [rows][576]
   const int* plan;                 // [n_seq + 1] tile prefix, then [G] first sequence of each CTA
   float scale_log2;                // log2(e) / sqrt(192)
   float* part_ml;                  // [G + n_seq][96][2]: reference max (raw logit units), sum
@@ -76,7 +78,7 @@ struct SplitParams {
 };
 
 // Walks the tiles of a CTA's range: sequence i, tile k of it.  The tile's
-// 64-row window ends at the sequence's end when the tile is the last one, so
+// BT-row window ends at the sequence's end when the tile is the last one, so
 // no row past the sequence (or the cache) is read; rows before the sequence
 // are masked (and rows before the cache read as zero).
 struct TileCursor {
@@ -130,7 +132,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   if (abort_flag) return;
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == PFULL || i == UFREE) ? 128 : 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == PFULL || i == UFREE || i == SFREE) ? 128 : 1);
     fence_mbar_init();
   }
   if (warp == 5) { tmem_alloc(smem_u32(&tmem_slot), 512); tmem_relinquish(); }
@@ -139,58 +141,70 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
+  // Ring order (producer and MMA thread walk it alike): the score-product
+  // pairs of tile 0; then, per tile t, the score-product pairs of tile t+1
+  // followed by the value-product pairs of tile t.
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmC); tma_prefetch_desc(&tmQ);
-      TileCursor cur = cursor(), pf = cursor();
+      TileCursor cq = cursor(), cp = cursor(), pf = cursor();
       int pf_t = 0;
       auto prefetch_upto = [&](int upto) {
         for (; pf_t < upto && pf_t < nt; ++pf_t) {
-          for (int x = 0; x < 9; ++x) tma_prefetch_l2_2d(&tmC, 64 * x, pf.row());
+          // A tile's rows are contiguous in the cache: bulk prefetches.
+          const int r0 = max(pf.row(), 0), r1 = pf.row() + BT;
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(p.cache + (size_t)r0 * WID);
+          for (uint32_t off = 0, n = (uint32_t)(r1 - r0) * WID * 2u; off < n; off += 16384u)
+            bulk_prefetch_l2(src + off, min(16384u, n - off));
           pf.next();
         }
       };
-      int seg = 0, lat_issued = 0, rope_issued = 0;
+      int u = 0, seg = 0, rope_issued = 0;
       bool ok = true;
+      auto load_pair = [&](int row, int pr) {
+        const uint32_t slot = (uint32_t)(u % NPS);
+        if (!mbar_wait(bar(LEMPTY + slot), ((uint32_t)(u / NPS) & 1u) ^ 1u, abort)) { ok = false; return; }
+        const uint32_t dst = sbase + OFF_PAIR + slot * PAIR;
+        mbar_arrive_expect_tx(bar(LFULL + slot), PAIR);
+        tma_load_2d(dst, &tmC, bar(LFULL + slot), 128 * pr, row);
+        tma_load_2d(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row);
+        ++u;
+      };
+      auto load_qk = [&](int t) {           // score-product items of tile t (cursor cq at t)
+        const int row = cq.row();
+        for (int pr = 0; pr < 4 && ok; ++pr) load_pair(row, pr);
+        if (!ok) return;
+        if (!mbar_wait(bar(REMPTY), ((uint32_t)t & 1u) ^ 1u, abort)) { ok = false; return; }
+        mbar_arrive_expect_tx(bar(RFULL), CSUB);
+        tma_load_2d(sbase + OFF_ROPE, &tmC, bar(RFULL), LAT, row);
+        ++rope_issued;
+      };
+      prefetch_upto(kPrefetchAhead);
+      mbar_arrive_expect_tx(bar(QFULL), 9 * QCH);
+      for (int c = 0; c < 9; ++c) tma_load_2d(sbase + OFF_Q + c * QCH, &tmQ, bar(QFULL), 64 * c, cq.i * HEADS);
+      load_qk(0);
       for (int t = 0; ok && t < nt; ++t) {
-        if (t == 0 || cur.k == 0) {
-          if (t > 0) {
+        const bool last = (t == nt - 1) || cq.last_of_seq();      // cq at tile t here
+        cq.next();
+        if (t + 1 < nt) {
+          if (last) {                        // tile t+1 starts another sequence: its q~
             ++seg;
             if (!mbar_wait(bar(QEMPTY), (uint32_t)(seg - 1) & 1u, abort)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar(QFULL), 9 * QCH);
+            for (int c = 0; c < 9; ++c) tma_load_2d(sbase + OFF_Q + c * QCH, &tmQ, bar(QFULL), 64 * c, cq.i * HEADS);
           }
-          mbar_arrive_expect_tx(bar(QFULL), 9 * QCH);
-          for (int c = 0; c < 9; ++c) tma_load_2d(sbase + OFF_Q + c * QCH, &tmQ, bar(QFULL), 64 * c, cur.i * HEADS);
+          load_qk(t + 1);
         }
-        prefetch_upto(t + 1 + kPrefetchAhead);
-        const int row = cur.row();
-        // Ring order = the order the MMA thread consumes: pairs 0, 1, the
-        // shared-key dims, pairs 2, 3.
-        for (int q = 0; q < 5 && ok; ++q) {
-          if (q == 2) {
-            if (!mbar_wait(bar(REMPTY), ((uint32_t)t & 1u) ^ 1u, abort)) { ok = false; break; }
-            mbar_arrive_expect_tx(bar(RFULL), CSUB);
-            tma_load_2d(sbase + OFF_ROPE, &tmC, bar(RFULL), LAT, row);
-            ++rope_issued;
-          } else {
-            const int pr = q < 2 ? q : q - 1;
-            const int u = 4 * t + pr;
-            const uint32_t slot = (uint32_t)(u % NLP);
-            if (!mbar_wait(bar(LEMPTY + slot), ((uint32_t)(u / NLP) & 1u) ^ 1u, abort)) { ok = false; break; }
-            const uint32_t dst = sbase + OFF_LAT + slot * PAIR;
-            mbar_arrive_expect_tx(bar(LFULL + slot), PAIR);
-            tma_load_2d(dst, &tmC, bar(LFULL + slot), 128 * pr, row);
-            tma_load_2d(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row);
-            lat_issued = u + 1;
-          }
-        }
-        cur.next();
+        const int row = cp.row();
+        for (int pr = 0; pr < 4 && ok; ++pr) load_pair(row, pr);
+        cp.next();
+        prefetch_upto(t + 2 + kPrefetchAhead);
       }
       // Never leave with copies in flight into this CTA's shared memory.
       mbar_wait_drain(bar(QFULL), (uint32_t)seg & 1u);
       if (rope_issued > 0) mbar_wait_drain(bar(RFULL), (uint32_t)(rope_issued - 1) & 1u);
-      for (int u = (lat_issued > NLP ? lat_issued - NLP : 0); u < lat_issued; ++u)
-        mbar_wait_drain(bar(LFULL + u % NLP), (uint32_t)(u / NLP) & 1u);
+      for (int v = (u > NPS ? u - NPS : 0); v < u; ++v) mbar_wait_drain(bar(LFULL + v % NPS), (uint32_t)(v / NPS) & 1u);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
@@ -198,82 +212,73 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
       constexpr uint32_t idQK = idesc_bf16_f32(128, BT, false, false);      // q~ (K-major) x tile (K-major)
       constexpr uint32_t idPV = idesc_bf16_f32(128, HEADS, true, false);    // tile^T (MN-major) x P^T (K-major)
       bool ok = true;
+      int u = 0;
       auto wait_ok = [&](int b, uint32_t ph) {
         ok = ok && mbar_wait(bar(b), ph, abort);
         if (ok) tc_fence_after();
         return ok;
       };
-      // Score product of tile t: q~ chunks 2pr, 2pr+1 against latent pair pr.
-      auto qk_pair = [&](int t, int pr, bool first) {
-        const int u = 4 * t + pr;
-        const uint32_t slot = (uint32_t)(u % NLP);
-        if (!wait_ok(LFULL + slot, (uint32_t)(u / NLP) & 1u)) return;
-        const uint32_t sb = sbase + OFF_LAT + slot * PAIR;
-        const uint32_t d = tmem + TM_S + (uint32_t)(t & 1) * BT;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(d, sdesc_sw128(sbase + OFF_Q + (uint32_t)(2 * pr + hf) * QCH + kk * 32u, 16, 1024),
-                   sdesc_sw128(sb + hf * CSUB + kk * 32u, 16, 1024), idQK, !(first && hf == 0 && kk == 0));
+      auto next_pair = [&]() -> uint32_t {    // wait for ring item u; returns its slot address
+        const uint32_t slot = (uint32_t)(u % NPS);
+        if (!wait_ok(LFULL + slot, (uint32_t)(u / NPS) & 1u)) return 0;
+        return sbase + OFF_PAIR + slot * PAIR;
       };
-      auto qk_rope = [&](int t) {
+      auto release_pair = [&]() { mma_commit(bar(LEMPTY + u % NPS)); ++u; };
+      auto qk = [&](int t) {
+        const uint32_t d = tmem + TM_S;
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t sb = next_pair();
+          if (!ok) return;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(d, sdesc_sw128(sbase + OFF_Q + (uint32_t)(2 * q + hf) * QCH + kk * 32u, 16, 1024),
+                     sdesc_sw128(sb + hf * CSUB + kk * 32u, 16, 1024), idQK, (q | hf | kk) != 0);
+          release_pair();
+        }
         if (!wait_ok(RFULL, (uint32_t)t & 1u)) return;
-        const uint32_t d = tmem + TM_S + (uint32_t)(t & 1) * BT;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(d, sdesc_sw128(sbase + OFF_Q + 8u * QCH + kk * 32u, 16, 1024),
                  sdesc_sw128(sbase + OFF_ROPE + kk * 32u, 16, 1024), idQK, true);
         mma_commit(bar(REMPTY));
-      };
-      // Value product of tile t, one 128-row latent block per pair; each
-      // pair slot is released as soon as its block is issued.
-      auto pv = [&](int t, bool fresh) {
-#pragma unroll 1
-        for (int b = 0; b < 4; ++b) {
-          const int u = 4 * t + b;
-          const uint32_t slot = (uint32_t)(u % NLP);
-          const uint32_t sb = sbase + OFF_LAT + slot * PAIR;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + TM_U + (uint32_t)b * HEADS, sdesc_sw128(sb + kk * 2048u, CSUB, 1024),
-                   sdesc_sw128(sbase + OFF_P + kk * 32u, 16, 1024), idPV, !(fresh && kk == 0));
-          mma_commit(bar(LEMPTY + slot));
-        }
-      };
-      TileCursor cur = cursor(), nxt = cursor();
-      nxt.next();
-      int seg = 0;
-      // Score product of the first tile.
-      if (wait_ok(QFULL, 0)) {
-        qk_pair(0, 0, true); qk_pair(0, 1, false); qk_rope(0); qk_pair(0, 2, false); qk_pair(0, 3, false);
         mma_commit(bar(SFULL));
-        if (nt == 1 || cur.last_of_seq()) mma_commit(bar(QEMPTY));
+      };
+      auto pv = [&](bool fresh) {
+        for (int b = 0; b < 4; ++b) {
+          const uint32_t sb = next_pair();
+          if (!ok) return;
+#pragma unroll
+          for (int kk = 0; kk < BT / 16; ++kk)
+            mma_ss(tmem + TM_U + (uint32_t)b * HEADS, sdesc_sw128(sb + kk * 2048u, CSUB, 1024),
+                   sdesc_sw128(sbase + OFF_P + (uint32_t)(kk >> 2) * QCH + (uint32_t)(kk & 3) * 32u, 16, 1024), idPV,
+                   !(fresh && kk == 0));
+          release_pair();
+        }
+        mma_commit(bar(PVDONE));
+      };
+      TileCursor cur = cursor();
+      int seg = 0;
+      if (wait_ok(QFULL, 0)) {
+        qk(0);
+        if (ok && ((nt == 1) || cur.last_of_seq())) mma_commit(bar(QEMPTY));
       }
       for (int t = 0; ok && t < nt; ++t) {
         const bool first = (t == 0) || cur.k == 0;
         const bool last = (t == nt - 1) || cur.last_of_seq();
-        const bool pre = (t + 1 < nt) && !last;           // tile t+1 continues this sequence
-        if (pre) { qk_pair(t + 1, 0, true); qk_pair(t + 1, 1, false); qk_rope(t + 1); }
+        cur.next();                          // now at tile t+1
+        if (t + 1 < nt) {
+          if (last && !wait_ok(QFULL, (uint32_t)(seg + 1) & 1u)) break;
+          // S is single-buffered: the softmax of tile t must have loaded it.
+          if (!wait_ok(SFREE, (uint32_t)t & 1u)) break;
+          qk(t + 1);
+          if (ok && ((t + 2 == nt) || cur.last_of_seq())) mma_commit(bar(QEMPTY));
+        }
         if (!wait_ok(PFULL, (uint32_t)t & 1u)) break;
         if (first && seg > 0 && !wait_ok(UFREE, (uint32_t)(seg - 1) & 1u)) break;
-        pv(t, first);
-        if (last) mma_commit(bar(SEGDONE));
-        if (t + 1 < nt) {
-          if (pre) {
-            qk_pair(t + 1, 2, false); qk_pair(t + 1, 3, false);
-          } else {
-            ++seg;
-            if (!wait_ok(QFULL, (uint32_t)seg & 1u)) break;
-            qk_pair(t + 1, 0, true); qk_pair(t + 1, 1, false); qk_rope(t + 1); qk_pair(t + 1, 2, false);
-            qk_pair(t + 1, 3, false);
-          }
-          if (!ok) break;
-          mma_commit(bar(SFULL + ((t + 1) & 1)));
-          if (t + 2 == nt || nxt.last_of_seq()) mma_commit(bar(QEMPTY));
-        }
-        cur.next();
-        nxt.next();
+        pv(first);
+        if (last) ++seg;
       }
       // Drain every MMA this thread issued before TMEM is released.
       mma_commit(bar(DRAIN));
@@ -290,35 +295,43 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
     const float thr_add = kRescaleLog2 / c;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    int seg = 0;
     TileCursor cur = cursor();
     // The loop runs the same named barriers in every thread whatever
     // happens, so a failed wait can never strand a warp in a barrier.
     for (int t = 0; t < nt; ++t) {
       const bool first = (t == 0) || cur.k == 0;
       const bool last = (t == nt - 1) || cur.last_of_seq();
-      if (ok) ok = mbar_wait(bar(SFULL + (t & 1)), (uint32_t)(t >> 1) & 1u, abort);
+      if (ok) ok = mbar_wait(bar(SFULL), (uint32_t)t & 1u, abort);
       ok = !bar_red_or(1, 128, !ok);
       float s[BT];
       bool need = false;
       float corr = 1.f, m_new = m_used;
       if (ok) {
         tc_fence_after();
-        const uint32_t ts = tmem + lane_off + TM_S + (uint32_t)(t & 1) * BT;
+        const uint32_t ts = tmem + lane_off + TM_S;
         tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&s[0]));
         tmem_ld32(ts + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
+        tmem_ld32(ts + 64u, *reinterpret_cast<float(*)[32]>(&s[64]));
         tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[0]));
         tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[32]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[64]));
+        tc_fence_before();
+        mbar_arrive(bar(SFREE));             // S may now be overwritten by the next tile's score product
         if (head) {
           const int w = cur.wrel();
           const int lo = cur.k * BT - w, hi = cur.L - w;   // valid columns [lo, hi)
           float pm[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
+          if (lo == 0 && hi >= BT) {
 #pragma unroll
-          for (int e = 0; e < BT; ++e) {
-            s[e] = (e >= lo && e < hi) ? s[e] : -INFINITY;
-            pm[e & 7] = fmaxf(pm[e & 7], s[e]);
+            for (int e = 0; e < BT; ++e) pm[e & 7] = fmaxf(pm[e & 7], s[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < BT; ++e) {
+              s[e] = (e >= lo && e < hi) ? s[e] : -INFINITY;
+              pm[e & 7] = fmaxf(pm[e & 7], s[e]);
+            }
           }
           const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
           need = mx > m_used + thr_add;                     // always on a piece's first tile
@@ -328,11 +341,30 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
         }
       }
       const bool resc = bar_red_or(1, 128, ok && head && need && !first);
+      // Probabilities first, into registers; P^T and U^T are touched only
+      // once the value product of tile t-1 has finished with them.
+      uint32_t pk[BT / 2];
+      if (ok && head) {
+        l *= corr;
+        m_used = m_new;
+        const float neg = -m_used * c;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < BT; e += 2) {
+          const float a0 = ex2(fmaf(s[e], c, neg)), a1 = ex2(fmaf(s[e + 1], c, neg));
+          ps[(e >> 1) & 7] += a0 + a1;
+          pk[e >> 1] = pack_bf16x2(a0, a1);
+        }
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      }
+      if (ok && t > 0) {
+        bool w = mbar_wait(bar(PVDONE), (uint32_t)(t - 1) & 1u, abort);
+        ok = __all_sync(0xffffffffu, w) != 0;
+        if (ok) tc_fence_after();
+      }
       if (ok && resc) {
-        // Rare: scale the U^T columns of the heads whose max moved.  The
-        // value product of tile t-1 has finished (it was issued before the
-        // score product of tile t), and that of tile t waits for this
-        // thread's arrival below.
+        // Rare: scale the U^T columns of the heads whose max moved (the
+        // value product of tile t waits for this thread's arrival below).
 #pragma unroll 1
         for (int b = 0; b < 4; ++b)
 #pragma unroll 1
@@ -348,23 +380,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
         tmem_wait_st();
       }
       if (ok && head) {
-        l *= corr;
-        m_used = m_new;
-        const float neg = -m_used * c;
-        const uint32_t prow = sbase + OFF_P + (uint32_t)x * 128u;
-        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // P^T row x: tokens 0-63 in the first sub-tile, 64-95 in the second.
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          float e8[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            e8[q] = ex2(fmaf(s[8 * cc + q], c, neg));
-            ps[q] += e8[q];
-          }
-          st_shared_v4(prow + ((uint32_t)(cc ^ (x & 7)) << 4), pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]),
-                       pack_bf16x2(e8[4], e8[5]), pack_bf16x2(e8[6], e8[7]));
+        for (int cc = 0; cc < BT / 8; ++cc) {
+          const uint32_t prow = sbase + OFF_P + (uint32_t)(cc >> 3) * QCH + (uint32_t)x * 128u;
+          st_shared_v4(prow + ((uint32_t)((cc & 7) ^ (x & 7)) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
+                       pk[4 * cc + 3]);
         }
-        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       }
       if (ok) {
         fence_proxy_async_smem();
@@ -372,8 +394,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
         mbar_arrive(bar(PFULL));
       }
       if (last) {
-        // End of this CTA's piece of sequence cur.i: write its partial.
-        bool w_ok = ok && mbar_wait(bar(SEGDONE), (uint32_t)seg & 1u, abort);
+        // End of this CTA's piece of sequence cur.i: write its partial once
+        // the value product of tile t has finished.
+        bool w_ok = ok && mbar_wait(bar(PVDONE), (uint32_t)t & 1u, abort);
         w_ok = __all_sync(0xffffffffu, w_ok) != 0;
         ok = ok && w_ok;
         if (ok) {
@@ -399,7 +422,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
         }
         m_used = -INFINITY;
         l = 0.f;
-        ++seg;
       }
       cur.next();
     }
