@@ -158,7 +158,8 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   const uint64_t rows = std::min<uint64_t>((uint64_t)n * (uint64_t)max_len, 0x7fffffffull);
   GMLA_TRY(make_map_2d(&mC, cache, tc_dec::WID, rows, tc_dec::BT));
   GMLA_TRY(make_map_2d(&mQ, q_abs, tc_dec::WID, (uint64_t)n * tc_dec::HEADS, tc_dec::HEADS));
-  tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256, tc_dec::ABS_SMEM, st>>>(
+  tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS, tc_dec::LAT / tc_dec::ABS_Q, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256,
+                          tc_dec::ABS_SMEM, st>>>(
       n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs, offs, G, plan);
   tc_dec::SplitParams sp;
   sp.n_seq = n; sp.G = G; sp.offs = offs; sp.plan = plan; sp.cache = static_cast<const bf*>(cache);
@@ -166,7 +167,8 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   sp.part_ml = part_ml; sp.part_u = part_u;
   tc_dec::decode_split_kernel<<<G, 192, tc_dec::SMEM_BYTES, st>>>(mC, mQ, sp);
   tc_dec::merge_kernel<<<(n * tc_dec::HEADS + 7) / 8, 256, 0, st>>>(n, G, plan, sp.scale_log2, part_ml, part_u, u_merged);
-  tc_dec::project_kernel<<<dim3(tc_dec::HEADS, (n + tc_dec::PRJ_SEQ - 1) / tc_dec::PRJ_SEQ), 256, tc_dec::PRJ_SMEM, st>>>(
+  tc_dec::project_kernel<<<dim3(tc_dec::HEADS, 128 / tc_dec::PRJ_Q, (n + tc_dec::PRJ_SEQ - 1) / tc_dec::PRJ_SEQ), 256,
+                           tc_dec::PRJ_SMEM, st>>>(
       n, u_merged, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate), static_cast<bf*>(O));
   note_launches(4);
   return check_launch();

@@ -495,28 +495,29 @@ __device__ void build_plan(int n_seq, const int* __restrict__ offs, int G, int* 
 }
 
 constexpr int ABS_SEQ = 64;                    // sequences per absorb block
+constexpr int ABS_Q = 128;                     // latent columns per absorb block
 constexpr int LDK = 136;                       // padded bf16 row of a 128-wide staged operand
-constexpr size_t ABS_SMEM = (size_t)(LAT + ABS_SEQ) * LDK * 2;
+constexpr size_t ABS_SMEM = (size_t)(ABS_Q + ABS_SEQ) * LDK * 2;
 
-// q~[i][h] = [q^C_h W_UK,h^T | q^S_h] in bf16.  Block = (head h, 64 sequences),
-// 8 warps.  W_UK,h (512 x 128, one 256-byte row segment per latent index)
-// and the block's q^C rows are staged in shared memory with 16-byte loads;
-// warp w computes latent columns [64w, 64w + 64).
-// Block (0, 0) also builds the split kernel's work plan.
+// q~[i][h] = [q^C_h W_UK,h^T | q^S_h] in bf16.  Block = (head h, 128 latent
+// columns, 64 sequences), 8 warps.  The block's rows of W_UK,h (128 x 128,
+// one 256-byte row segment per latent index) and its q^C rows are staged in
+// shared memory with 16-byte loads; warp w computes 16 latent columns.
+// Block (0, 0, 0) also builds the split kernel's work plan.
 __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ W_UKV,
                                                      __nv_bfloat16* __restrict__ q_abs, const int* __restrict__ offs,
                                                      int G, int* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t asm_[];
-  __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(asm_);      // [512][LDK]: W_UK,h[latent][k]
-  __nv_bfloat16* As = Ws + LAT * LDK;                               // [64][LDK]: q^C[i][k]
-  const int h = blockIdx.x, i0 = blockIdx.y * ABS_SEQ;
+  __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(asm_);      // [128][LDK]: W_UK,h[latent][k]
+  __nv_bfloat16* As = Ws + ABS_Q * LDK;                             // [64][LDK]: q^C[i][k]
+  const int h = blockIdx.x, n0 = blockIdx.y * ABS_Q, i0 = blockIdx.z * ABS_SEQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   constexpr size_t ldw = (size_t)HEADS * 256;
-  if (blockIdx.x == 0 && blockIdx.y == 0) build_plan(n_seq, offs, G, plan);
-  for (int e = threadIdx.x; e < LAT * 16; e += blockDim.x) {
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) build_plan(n_seq, offs, G, plan);
+  for (int e = threadIdx.x; e < ABS_Q * 16; e += blockDim.x) {
     const int n = e >> 4, c = e & 15;
-    cp_async16(Ws + n * LDK + c * 8, W_UKV + (size_t)n * ldw + (size_t)h * 256 + c * 8);
+    cp_async16(Ws + n * LDK + c * 8, W_UKV + (size_t)(n0 + n) * ldw + (size_t)h * 256 + c * 8);
   }
   for (int e = threadIdx.x; e < ABS_SEQ * 16; e += blockDim.x) {
     const int r = e >> 4, c = e & 15, i = i0 + r;
@@ -527,22 +528,22 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
   __syncthreads();
 #pragma unroll 1
   for (int mt = 0; mt < ABS_SEQ / 16; ++mt) {
-    float acc[8][4] = {};
+    float acc[2][4] = {};
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const int k0 = kk * 16 + 2 * t;
       const __nv_bfloat16* ar = As + (mt * 16 + g) * LDK + k0;
       const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDK), lds32(ar + 8), lds32(ar + 8 * LDK + 8)};
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const __nv_bfloat16* br = Ws + (warp * 64 + nt * 8 + g) * LDK + k0;
+      for (int nt = 0; nt < 2; ++nt) {
+        const __nv_bfloat16* br = Ws + (warp * 16 + nt * 8 + g) * LDK + k0;
         mma16816(acc[nt], a, lds32(br), lds32(br + 8));
       }
     }
     const int ra = i0 + mt * 16 + g, rb = ra + 8;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int col = warp * 64 + nt * 8 + 2 * t;
+    for (int nt = 0; nt < 2; ++nt) {
+      const int col = n0 + warp * 16 + nt * 8 + 2 * t;
       if (ra < n_seq)
         *reinterpret_cast<__nv_bfloat162*>(q_abs + ((size_t)ra * HEADS + h) * WID + col) = __floats2bfloat162_rn(acc[nt][0], acc[nt][1]);
       if (rb < n_seq)
@@ -550,6 +551,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
     }
   }
   // q^S passes through unchanged: 64 values = 8 x 16 bytes per sequence.
+  if (blockIdx.y != 0) return;
   for (int e = threadIdx.x; e < ABS_SEQ * 8; e += blockDim.x) {
     const int i = i0 + (e >> 3), c = e & 7;
     if (i < n_seq)
@@ -609,25 +611,28 @@ __global__ void __launch_bounds__(256) merge_kernel(int n_seq, int G, const int*
 }
 
 constexpr int PRJ_SEQ = 64;                    // sequences per projection block
+constexpr int PRJ_Q = 32;                      // output columns per projection block
 constexpr int LDU = LAT + 8;                   // padded bf16 row of the staged latent tile
-constexpr size_t PRJ_SMEM = (size_t)LAT * LDK * 2 + (size_t)PRJ_SEQ * LDU * 2;
+constexpr int LDWQ = PRJ_Q + 8;                // padded bf16 row of the staged W_UV,h columns
+constexpr size_t PRJ_SMEM = (size_t)LAT * LDWQ * 2 + (size_t)PRJ_SEQ * LDU * 2;
 
-// o[i][h] = u[i][h] W_UV,h (* sigmoid(g)).  Block = (head h, 64 sequences),
-// 8 warps; warp w owns output columns [16w, 16w + 16).  W_UV,h (512 x 128,
-// row-major) and the block's merged latents are staged with cp.async; W_UV,h
-// feeds the MMA through transposing matrix loads.
+// o[i][h] = u[i][h] W_UV,h (* sigmoid(g)).  Block = (head h, 32 output
+// columns, 64 sequences), 8 warps; warp w owns 8 output columns of 32
+// sequences.  The block's columns of W_UV,h (512 x 32, row-major) and its
+// merged latents are staged with cp.async; W_UV,h feeds the MMA through
+// transposing matrix loads.
 __global__ void __launch_bounds__(256) project_kernel(int n_seq, const __nv_bfloat16* __restrict__ u_in,
                                                       const __nv_bfloat16* __restrict__ W_UKV,
                                                       const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ O) {
   extern __shared__ __align__(16) uint8_t csm[];
-  __nv_bfloat16* Wv = reinterpret_cast<__nv_bfloat16*>(csm);                    // [512][LDK]
-  __nv_bfloat16* U = Wv + LAT * LDK;                                             // [64][LDU]
-  const int h = blockIdx.x, i0 = blockIdx.y * PRJ_SEQ;
+  __nv_bfloat16* Wv = reinterpret_cast<__nv_bfloat16*>(csm);                    // [512][LDWQ]
+  __nv_bfloat16* U = Wv + LAT * LDWQ;                                            // [64][LDU]
+  const int h = blockIdx.x, q0 = blockIdx.y * PRJ_Q, i0 = blockIdx.z * PRJ_SEQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t = lane & 3;
   constexpr size_t ldw = (size_t)HEADS * 256;
-  for (int e = threadIdx.x; e < LAT * 16; e += blockDim.x) {
-    const int k = e >> 4, c = e & 15;
-    cp_async16(Wv + k * LDK + c * 8, W_UKV + (size_t)k * ldw + (size_t)h * 256 + 128 + c * 8);
+  for (int e = threadIdx.x; e < LAT * (PRJ_Q / 8); e += blockDim.x) {
+    const int k = e / (PRJ_Q / 8), c = e % (PRJ_Q / 8);
+    cp_async16(Wv + k * LDWQ + c * 8, W_UKV + (size_t)k * ldw + (size_t)h * 256 + 128 + q0 + c * 8);
   }
   for (int e = threadIdx.x; e < PRJ_SEQ * (LAT / 8); e += blockDim.x) {
     const int r = e / (LAT / 8), c = e % (LAT / 8), i = i0 + r;
@@ -636,42 +641,37 @@ __global__ void __launch_bounds__(256) project_kernel(int n_seq, const __nv_bflo
   }
   cp_async_wait_all();
   __syncthreads();
-  float acc[4][2][4] = {};
+  const int nt = warp & 3, mt0 = (warp >> 2) * 2;
+  float acc[2][4] = {};
 #pragma unroll 4
   for (int kk = 0; kk < LAT / 16; ++kk) {
     const int k0 = kk * 16;
-    uint32_t bf[2][2];
+    uint32_t b0, b1;
+    ldsm_x2_trans(b0, b1, Wv + (k0 + (lane & 15)) * LDWQ + nt * 8);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-      ldsm_x2_trans(bf[nt][0], bf[nt][1], Wv + (k0 + (lane & 15)) * LDK + warp * 16 + nt * 8);
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
-      const __nv_bfloat16* ar = U + (mt * 16 + gq) * LDU + k0 + 2 * t;
+    for (int m = 0; m < 2; ++m) {
+      const __nv_bfloat16* ar = U + ((mt0 + m) * 16 + gq) * LDU + k0 + 2 * t;
       const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDU), lds32(ar + 8), lds32(ar + 8 * LDU + 8)};
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) mma16816(acc[mt][nt], a, bf[nt][0], bf[nt][1]);
+      mma16816(acc[m], a, b0, b1);
     }
   }
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
+  for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int i = i0 + mt * 16 + gq + 8 * hr;
-        if (i >= n_seq) continue;
-        const int col = warp * 16 + nt * 8 + 2 * t;
-        const size_t idx = ((size_t)i * HEADS + h) * 128 + col;
-        float o0 = acc[mt][nt][2 * hr], o1 = acc[mt][nt][2 * hr + 1];
-        if (g) {
-          const float2 gv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(g + idx));
-          o0 *= 1.f / (1.f + __expf(-gv.x));
-          o1 *= 1.f / (1.f + __expf(-gv.y));
-        }
-        *reinterpret_cast<__nv_bfloat162*>(O + idx) = __floats2bfloat162_rn(o0, o1);
+    for (int hr = 0; hr < 2; ++hr) {
+      const int i = i0 + (mt0 + m) * 16 + gq + 8 * hr;
+      if (i >= n_seq) continue;
+      const int col = q0 + nt * 8 + 2 * t;
+      const size_t idx = ((size_t)i * HEADS + h) * 128 + col;
+      float o0 = acc[m][2 * hr], o1 = acc[m][2 * hr + 1];
+      if (g) {
+        const float2 gv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(g + idx));
+        o0 *= 1.f / (1.f + __expf(-gv.x));
+        o1 *= 1.f / (1.f + __expf(-gv.y));
       }
+      *reinterpret_cast<__nv_bfloat162*>(O + idx) = __floats2bfloat162_rn(o0, o1);
+    }
 }
-
 
 
 inline size_t workspace_bytes(int n) {
