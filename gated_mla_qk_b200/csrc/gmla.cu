@@ -228,7 +228,12 @@ static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfl
   GMLA_TRY(make_map_2d(&mB, B, (uint64_t)N, (uint64_t)K, tc_gemm::BK));
   tc_gemm::Params p;
   p.M = M; p.N = N; p.K = K; p.C = C; p.KC = KC; p.V = V; p.H = H; p.mode = mode;
-  const unsigned grid = (unsigned)((N + tc_gemm::BN - 1) / tc_gemm::BN) * (unsigned)((M + tc_gemm::BM - 1) / tc_gemm::BM);
+  // Persistent: one CTA per SM (never more CTAs than output tiles).
+  int dev = 0, sms = 0;
+  GMLA_TRY(cuda_status(cudaGetDevice(&dev)));
+  GMLA_TRY(cuda_status(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)));
+  const long long tiles = (long long)((N + tc_gemm::BN - 1) / tc_gemm::BN) * ((M + tc_gemm::BM - 1) / tc_gemm::BM);
+  const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms));
   tc_gemm::gemm_kernel<<<grid, 192, tc_gemm::SMEM_BYTES, st>>>(mA, mB, p);
   note_launches(1);
   return check_launch();

@@ -3,12 +3,15 @@
 // c^Q = x W_DQ, q = c^Q W_UQ, [c^KV k^S] = x W_DKV, [k^C v] = c^KV W_UKV).
 //
 // C[M][N] = A[M][K] B[K][N], all row-major; fp32 accumulation in TMEM.
-// One CTA per 128 x 256 output tile.  A tiles (128 x 64, K-major) and B tiles
-// (64 x 256, N contiguous = MN-major) stream through a 4-stage TMA ring; one
-// thread issues tcgen05.mma (M=128, N=256, K=16) into a 256-column TMEM
-// accumulator; four epilogue warps read it back with tcgen05.ld and store
-// bf16.  The epilogue either writes C row-major or, for the key/value
-// up-projection, splits each 256-column tile (= one head) into K^C and V.
+// Persistent: one CTA per SM walks the 128 x 256 output tiles (tile index
+// advancing by the grid size).  A tiles (128 x 64, K-major) and B tiles
+// (64 x 256, N contiguous = MN-major) stream through a 4-stage TMA ring that
+// runs on across tile boundaries; one thread issues tcgen05.mma (M=128,
+// N=256, K=16) into one of two 256-column TMEM accumulators, so the four
+// epilogue warps read tile j back (tcgen05.ld, bf16 stores) while the MMAs
+// of tile j+1 run.  The epilogue either writes C row-major or, for the
+// key/value up-projection, splits each 256-column tile (= one head) into K^C
+// and V.
 #pragma once
 
 #include "sm100.cuh"
@@ -26,7 +29,7 @@ constexpr uint32_t STAGE = A_BYTES + B_BYTES;             // 48 KB
 constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
 
-enum Bar { FULL = 0, EMPTY = NSTAGE, ACC = 2 * NSTAGE, NBAR = 2 * NSTAGE + 1 };
+enum Bar { FULL = 0, EMPTY = NSTAGE, ACCF = 2 * NSTAGE, ACCE = ACCF + 2, DRAIN = ACCE + 2, NBAR = DRAIN + 1 };
 
 struct Params {
   int M, N, K;
@@ -47,18 +50,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   volatile int* abort = &abort_flag;
   auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (p.N + BN - 1) / BN;
-  const int tn = blockIdx.x % n_tiles, tm = blockIdx.x / n_tiles;
+  const int n_tiles_n = (p.N + BN - 1) / BN;
+  const int n_tiles = n_tiles_n * ((p.M + BM - 1) / BM);
   const int nk = (p.K + BK - 1) / BK;
 
   if (threadIdx.x == 0) abort_flag = device_error_pending() ? 1 : 0;
   __syncthreads();
   if (abort_flag) return;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == ACCE || i == ACCE + 1) ? 128 : 1);
     fence_mbar_init();
   }
-  if (warp == 1) { tmem_alloc(smem_u32(&tmem_slot), 256); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(smem_u32(&tmem_slot), 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -67,56 +70,74 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
-      int issued = 0;
-      for (int k = 0; k < nk; ++k) {
-        const uint32_t s = k % NSTAGE, ph = (k / NSTAGE) & 1;
-        if (!mbar_wait(bar(EMPTY + s), ph ^ 1u, abort)) break;
-        const uint32_t st = sbase + s * STAGE;
-        mbar_arrive_expect_tx(bar(FULL + s), STAGE);
-        tma_load_2d(st, &tmA, bar(FULL + s), k * BK, tm * BM);
-        for (int c = 0; c < 4; ++c) tma_load_2d(st + A_BYTES + c * BSUB, &tmB, bar(FULL + s), tn * BN + 64 * c, k * BK);
-        ++issued;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+        const int tn = tile % n_tiles_n, tm = tile / n_tiles_n;
+        for (int k = 0; k < nk; ++k, ++it) {
+          const uint32_t s = it % NSTAGE, ph = (it / NSTAGE) & 1;
+          if (!mbar_wait(bar(EMPTY + s), ph ^ 1u, abort)) { ok = false; break; }
+          const uint32_t st = sbase + s * STAGE;
+          mbar_arrive_expect_tx(bar(FULL + s), STAGE);
+          tma_load_2d(st, &tmA, bar(FULL + s), k * BK, tm * BM);
+          for (int c = 0; c < 4; ++c) tma_load_2d(st + A_BYTES + c * BSUB, &tmB, bar(FULL + s), tn * BN + 64 * c, k * BK);
+        }
       }
-      for (int k = (issued > NSTAGE ? issued - NSTAGE : 0); k < issued; ++k)
-        mbar_wait_drain(bar(FULL + k % NSTAGE), (k / NSTAGE) & 1);
+      for (int q = (it > NSTAGE ? it - NSTAGE : 0); q < it; ++q)
+        mbar_wait_drain(bar(FULL + q % NSTAGE), (q / NSTAGE) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, true);   // A K-major, B MN-major
-      for (int k = 0; k < nk; ++k) {
-        const uint32_t s = k % NSTAGE, ph = (k / NSTAGE) & 1;
-        if (!mbar_wait(bar(FULL + s), ph, abort)) break;
+      int it = 0, j = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++j) {
+        const int acc = j & 1;
+        // Accumulator acc was last used by tile j-2: its epilogue must be done.
+        if (j >= 2 && !(ok = mbar_wait(bar(ACCE + acc), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort))) break;
         tc_fence_after();
-        const uint32_t st = sbase + s * STAGE;
+        const uint32_t d = tmem + 256u * (uint32_t)acc;
+        for (int k = 0; k < nk; ++k, ++it) {
+          const uint32_t s = it % NSTAGE, ph = (it / NSTAGE) & 1;
+          if (!(ok = mbar_wait(bar(FULL + s), ph, abort))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + s * STAGE;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ss(tmem, sdesc_sw128(st + kk * 32, 16, 1024), sdesc_sw128(st + A_BYTES + kk * 2048, BSUB, 1024), idesc,
-                 (k > 0 || kk > 0));
-        mma_commit(bar(EMPTY + s));
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_ss(d, sdesc_sw128(st + kk * 32, 16, 1024), sdesc_sw128(st + A_BYTES + kk * 2048, BSUB, 1024), idesc,
+                   (k > 0 || kk > 0));
+          mma_commit(bar(EMPTY + s));
+        }
+        if (!ok) break;
+        mma_commit(bar(ACCF + acc));
       }
-      mma_commit(bar(ACC));
-      mbar_wait_drain(bar(ACC), 0);
+      mma_commit(bar(DRAIN));
+      mbar_wait_drain(bar(DRAIN), 0);
     }
     __syncwarp();
   } else {
     // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) .. + 31
     const int sub = warp & 3;
-    const int row = tm * BM + sub * 32 + lane;
-    const bool ok = mbar_wait(bar(ACC), 0, abort);
-    if (__all_sync(0xffffffffu, ok)) {
+    int j = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
+      const int acc = j & 1;
+      const bool w = mbar_wait(bar(ACCF + acc), (uint32_t)(j >> 1) & 1u, abort);
+      if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16);
+      const int tn = tile % n_tiles_n, tm = tile / n_tiles_n;
+      const int row = tm * BM + sub * 32 + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + 256u * (uint32_t)acc;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(taddr + 32u * c, v);
-        tmem_wait_ld();
+        tmem_wait_ld_dep(v);
         const int col0 = tn * BN + 32 * c;
         if (row < p.M && col0 < p.N) {
           __nv_bfloat16* dst;
           if (p.mode == 1) {
-            const int h = col0 / 256, j = col0 % 256;
-            dst = (j < 128) ? p.KC + ((size_t)row * p.H + h) * 128 + j : p.V + ((size_t)row * p.H + h) * 128 + (j - 128);
+            const int h = col0 / 256, jj = col0 % 256;
+            dst = (jj < 128) ? p.KC + ((size_t)row * p.H + h) * 128 + jj : p.V + ((size_t)row * p.H + h) * 128 + (jj - 128);
           } else {
             dst = p.C + (size_t)row * p.N + col0;
           }
@@ -133,13 +154,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(bar(ACCE + acc));
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
