@@ -147,7 +147,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);   // Q (K-major) x K (K-major)
-      constexpr uint32_t idO = idesc_bf16_f32(128, 128, false, true);    // P (K-major) x V (MN-major)
+      constexpr uint32_t idO = idesc_bf16_f32(128, 128, false, true);    // P (TMEM) x V (MN-major)
       const uint32_t tS0 = tmem, tO = tmem + 256;
       uint32_t u = 0;
       bool ok = mbar_wait(bar(QFULL), 0, abort);
@@ -180,11 +180,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!mbar_wait(bar(KVFULL + slot), ph, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t vbase = sbase + OFF_RING + slot * 3 * SUB;
+        // P_j sits in the first 64 columns of S buffer (j & 1), two bf16 per column.
+        const uint32_t tP = tS0 + (uint32_t)(j & 1) * 128u;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint32_t pa = sbase + OFF_P + (uint32_t)(i >> 2) * SUB + (uint32_t)(i & 3) * 32u;
           const uint32_t vb = vbase + (uint32_t)i * 2048u;     // 16 keys x 128 B rows
-          mma_ss(tO, sdesc_sw128(pa, 16, 1024), sdesc_sw128(vb, SUB, 1024), idO, (j > 0 || i > 0));
+          mma_ts(tO, tP + 8u * (uint32_t)i, sdesc_sw128(vb, SUB, 1024), idO, (j > 0 || i > 0));
         }
         mma_commit(bar(PVDONE));
         mma_commit(bar(KVEMPTY + slot));
@@ -220,18 +221,35 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         float (&chunk)[32] = *reinterpret_cast<float(*)[32]>(&s[32 * k]);
         tmem_ld32(tS_row + (uint32_t)buf * 128u + 32u * k, chunk);
       }
-      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[32 * k]));
       if (j == qt) {                           // diagonal tile: key column > query row is masked
 #pragma unroll
         for (int k = 0; k < 128; ++k) s[k] = (k > r) ? -INFINITY : s[k];
       }
-      float mx = s[0];
+      // Row max with eight independent accumulators (a single chain would
+      // serialise 127 dependent max operations).
+      float pm[8];
 #pragma unroll
-      for (int k = 1; k < 128; ++k) mx = fmaxf(mx, s[k]);
+      for (int q = 0; q < 8; ++q) pm[q] = s[q];
+#pragma unroll
+      for (int k = 8; k < 128; ++k) pm[k & 7] = fmaxf(pm[k & 7], s[k]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       true_max = fmaxf(true_max, mx);
       const bool need = (m_used == -INFINITY) || ((mx - m_used) * c > kRescaleLog2);
       const float m_new = need ? fmaxf(m_used, mx) : m_used;
       const float corr = need ? ex2((m_used - m_new) * c) : 1.f;
+      // Probabilities into registers first (bf16 pairs), so that they are
+      // computed while the P.V product of tile j-1 still reads the P buffer.
+      const float neg = -m_new * c;
+      uint32_t pk[64];
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < 128; e += 2) {
+        const float a0 = ex2(fmaf(s[e], c, neg)), a1 = ex2(fmaf(s[e + 1], c, neg));
+        ps[(e >> 1) & 7] += a0 + a1;
+        pk[e >> 1] = pack_bf16x2(a0, a1);
+      }
       if (j > 0) {
         if (!wait_warp(PVDONE, (uint32_t)(j - 1) & 1u)) { ok = false; break; }
         tc_fence_after();
@@ -240,7 +258,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int k = 0; k < 4; ++k) {
             float o[32];
             tmem_ld32(tO_row + 32u * k, o);
-            tmem_wait_ld();
+            tmem_wait_ld_dep(o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= corr;
             tmem_st32(tO_row + 32u * k, o);
@@ -248,20 +266,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tmem_wait_st();
         }
       }
-      l *= corr;
+      l = l * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
       m_used = m_new;
-      const float neg = -m_used * c;
-      const uint32_t prow = sbase + OFF_P + (uint32_t)r * 128u;
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        float e8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { e8[e] = ex2(fmaf(s[8 * cc + e], c, neg)); l += e8[e]; }
-        const uint32_t addr = prow + (uint32_t)(cc >> 3) * SUB + ((uint32_t)((cc & 7) ^ (r & 7)) << 4);
-        st_shared_v4(addr, pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]), pack_bf16x2(e8[4], e8[5]),
-                     pack_bf16x2(e8[6], e8[7]));
-      }
-      fence_proxy_async_smem();
+      // P into TMEM over the first 64 columns of its own S buffer (S has been
+      // read; the score product that next writes this buffer is issued after
+      // this tile's P.V product).
+      tmem_st32u(tS_row + (uint32_t)buf * 128u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+      tmem_st32u(tS_row + (uint32_t)buf * 128u + 32u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(PFULL));
     }
