@@ -178,12 +178,15 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
 // Attention forward dispatch
 // ---------------------------------------------------------------------------
 static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const void* KC, const void* kS,
-                       const void* V, const void* gate, void* O, float* maxlogit, cudaStream_t st) {
+                       const void* V, const void* gate, void* O, bool out_f32, float* maxlogit, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)tc_attn::SMEM_BYTES);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tc_attn::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_status(attr_err);
   CUtensorMap mQ, mKC, mKS, mV;
@@ -195,13 +198,14 @@ static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const vo
   tc_attn::Params p;
   p.B = B; p.T = T; p.H = H; p.n_qtiles = (T + tc_attn::BM - 1) / tc_attn::BM;
   p.g = static_cast<const __nv_bfloat16*>(gate);
-  p.O = static_cast<__nv_bfloat16*>(O);
+  p.O = O;
   p.maxlogit = maxlogit;
   p.scale = 1.f / std::sqrt(192.f);
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   simt::fill_kernel<<<(H + 127) / 128, 128, 0, st>>>(maxlogit, H, -INFINITY);
   const unsigned grid = (unsigned)p.n_qtiles * (unsigned)H * (unsigned)B;
-  tc_attn::attn_fwd_kernel<<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, p);
+  if (out_f32) tc_attn::attn_fwd_kernel<true><<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, p);
+  else tc_attn::attn_fwd_kernel<false><<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, p);
   note_launches(2);
   return check_launch();
 }
@@ -387,7 +391,7 @@ int mla_attn_fwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void*
   cudaStream_t st = as_stream(stream);
   if (dtype == GMLA_BF16 && is_k3_head_geometry(g)) {
     if ((long long)B * T * g->H * 192 >= (1LL << 40)) return GMLA_EUNSUPPORTED;
-    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, maxlogit, st);
+    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, false, maxlogit, st);
   }
   if (g->d_c + g->d_s > 256 || g->d_v > simt::kAttnMaxDV) return GMLA_EUNSUPPORTED;
   if (dtype == GMLA_F32)
@@ -396,6 +400,30 @@ int mla_attn_fwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void*
   using bf = __nv_bfloat16;
   return simt::attn_fwd<bf>(B, T, g->H, g->d_c, g->d_s, g->d_v, (const bf*)Q, (const bf*)KC, (const bf*)kS,
                             (const bf*)V, (const bf*)gate, (bf*)O, maxlogit, st);
+}
+
+// ---------------------------------------------------------------------------
+// Training variant: the same forward with o kept in fp32.
+int mla_attn_fwd_train(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void* Q, const void* KC,
+                       const void* kS, const void* V, const void* gate, float* O, float* maxlogit, void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  if (B <= 0 || T <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(Q); GMLA_REQUIRE(KC); GMLA_REQUIRE(V); GMLA_REQUIRE(O); GMLA_REQUIRE(maxlogit);
+  if (g->d_s > 0) GMLA_REQUIRE(kS);
+  GMLA_OPTIONAL(gate);
+  cudaStream_t st = as_stream(stream);
+  if (dtype == GMLA_BF16 && is_k3_head_geometry(g)) {
+    if ((long long)B * T * g->H * 192 >= (1LL << 40)) return GMLA_EUNSUPPORTED;
+    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, true, maxlogit, st);
+  }
+  if (g->d_c + g->d_s > 256 || g->d_v > simt::kAttnMaxDV) return GMLA_EUNSUPPORTED;
+  if (dtype == GMLA_F32)
+    return simt::attn_fwd<float>(B, T, g->H, g->d_c, g->d_s, g->d_v, (const float*)Q, (const float*)KC,
+                                 (const float*)kS, (const float*)V, (const float*)gate, O, maxlogit, st);
+  using bf = __nv_bfloat16;
+  return simt::attn_fwd<bf, float>(B, T, g->H, g->d_c, g->d_s, g->d_v, (const bf*)Q, (const bf*)KC, (const bf*)kS,
+                                   (const bf*)V, (const bf*)gate, O, maxlogit, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -144,10 +144,10 @@ __global__ void norm_kv_rows_kernel(const T* __restrict__ ckv_ks, int kv_lora, i
 // ---------------------------------------------------------------------------
 constexpr int kAttnBQ = 16, kAttnBK = 32, kAttnMaxDV = 256;
 
-template <typename T>
+template <typename T, typename TO = T>
 __global__ void __launch_bounds__(128) attn_fwd_kernel(
     int T_, int H, int d_c, int d_s, int d_v, const T* __restrict__ Q, const T* __restrict__ KC,
-    const T* __restrict__ kS, const T* __restrict__ V, const T* __restrict__ g, T* __restrict__ O,
+    const T* __restrict__ kS, const T* __restrict__ V, const T* __restrict__ g, TO* __restrict__ O,
     float* __restrict__ maxlogit, float scale) {
   extern __shared__ float smem[];
   const int d_qk = d_c + d_s;
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(
       float o = acc[k] * inv_l;
       const size_t idx = ((size_t)b * T_ + t_row) * H * d_v + (size_t)h * d_v + c;
       if (g) o *= 1.f / (1.f + expf(-ld(g + idx)));
-      O[idx] = cvt<T>(o);
+      O[idx] = cvt<TO>(o);
     }
   }
   if (lane8 == 0) sMax[r] = (t_row < T_) ? m_run : -INFINITY;
@@ -250,17 +250,17 @@ inline size_t attn_smem_bytes(int d_qk, int d_v) {
   return sizeof(float) * (size_t)(kAttnBQ * d_qk + kAttnBK * (d_qk + 1) + kAttnBK * d_v + kAttnBQ * (kAttnBK + 1));
 }
 
-template <typename T>
+template <typename T, typename TO = T>
 inline int attn_fwd(int B, int T_, int H, int d_c, int d_s, int d_v, const T* Q, const T* KC, const T* kS,
-                    const T* V, const T* g, T* O, float* maxlogit, cudaStream_t st) {
+                    const T* V, const T* g, TO* O, float* maxlogit, cudaStream_t st) {
   const size_t smem = attn_smem_bytes(d_c + d_s, d_v);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<T, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_status(e);
   }
   fill_kernel<<<(H + 127) / 128, 128, 0, st>>>(maxlogit, H, -INFINITY);
   dim3 grid((T_ + kAttnBQ - 1) / kAttnBQ, H, B);
-  attn_fwd_kernel<T><<<grid, 128, smem, st>>>(T_, H, d_c, d_s, d_v, Q, KC, kS, V, g, O, maxlogit,
+  attn_fwd_kernel<T, TO><<<grid, 128, smem, st>>>(T_, H, d_c, d_s, d_v, Q, KC, kS, V, g, O, maxlogit,
                                               1.f / sqrtf((float)(d_c + d_s)));
   note_launches(2);
   return check_launch();

@@ -51,7 +51,7 @@ constexpr float kRescaleLog2 = 8.f;   // rescale O when the row max grows by > 2
 struct Params {
   int B, T, H, n_qtiles;
   const __nv_bfloat16* g;   // [B][T][H*128] or nullptr
-  __nv_bfloat16* O;         // [B][T][H*128]
+  void* O;                  // [B][T][H*128], bf16 or (training variant) fp32
   float* maxlogit;          // [H]
   float scale;              // 1/sqrt(192)
   float scale_log2;         // log2(e)/sqrt(192)
@@ -59,6 +59,11 @@ struct Params {
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
 
+// OUT_F32: the output is kept in fp32 (the training variant of "Gated MLA
+// et NoPE", "Un détail de précision numérique": no rounding of o to bf16).
+// The epilogue stores straight from registers, so no output tile occupies
+// shared memory in either variant.
+template <bool OUT_F32>
 __global__ void __launch_bounds__(192, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKC,
                 const __grid_constant__ CUtensorMap tmKS, const __grid_constant__ CUtensorMap tmV, Params p) {
@@ -286,10 +291,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int k = 0; k < 4; ++k) {
         float o[32];
         tmem_ld32(tO_row + 32u * k, o);
-        tmem_wait_ld();
+        tmem_wait_ld_dep(o);
         if (valid) {
           const uint4* gp = reinterpret_cast<const uint4*>(p.g + row_off + 32 * k);
-          uint4* op = reinterpret_cast<uint4*>(p.O + row_off + 32 * k);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             float gate[8];
@@ -306,12 +310,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
               for (int e = 0; e < 8; ++e) gate[e] = 1.f;
             }
-            uint4 ov;
-            ov.x = pack_bf16x2(o[8 * v + 0] * inv_l * gate[0], o[8 * v + 1] * inv_l * gate[1]);
-            ov.y = pack_bf16x2(o[8 * v + 2] * inv_l * gate[2], o[8 * v + 3] * inv_l * gate[3]);
-            ov.z = pack_bf16x2(o[8 * v + 4] * inv_l * gate[4], o[8 * v + 5] * inv_l * gate[5]);
-            ov.w = pack_bf16x2(o[8 * v + 6] * inv_l * gate[6], o[8 * v + 7] * inv_l * gate[7]);
-            op[v] = ov;
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = o[8 * v + e] * inv_l * gate[e];
+            if constexpr (OUT_F32) {
+              float4* op = reinterpret_cast<float4*>(static_cast<float*>(p.O) + row_off + 32 * k) + 2 * v;
+              op[0] = make_float4(y[0], y[1], y[2], y[3]);
+              op[1] = make_float4(y[4], y[5], y[6], y[7]);
+            } else {
+              uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.O) + row_off + 32 * k);
+              op[v] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                                 pack_bf16x2(y[6], y[7]));
+            }
           }
         }
       }

@@ -105,6 +105,21 @@ int mla_attn_fwd(const gmla_geom* geom, gmla_dtype dtype, int B, int T,
                  const void* g, void* O, float* maxlogit, void* stream);
 
 /*
+ * mla_attn_fwd_train — the same forward with the output kept in fp32, the
+ * training form of "Gated MLA et NoPE", "Un détail de précision numérique"
+ * (the attention output stays in FP32 during training, so no biased
+ * rounding of o to bf16).  Arguments, layouts, ownership and errors are those
+ * of mla_attn_fwd except:
+ *   O [B][T][H*d_v] float32 (written) whatever `dtype` is.
+ * bf16 with d_c=128, d_s=64, d_v=128 runs the tcgen05/TMA kernel (its epilogue
+ * stores from registers: no output tile is staged in shared memory); other
+ * shapes and fp32 inputs run the CUDA-core kernel with fp32 output.
+ */
+int mla_attn_fwd_train(const gmla_geom* geom, gmla_dtype dtype, int B, int T,
+                       const void* Q, const void* KC, const void* kS, const void* V,
+                       const void* g, float* O, float* maxlogit, void* stream);
+
+/*
  * qkclip_rescale — QK-Clip applied to the weights, in place.
  * "Anthology of the SOTA" record SOTA-131, "Source": after a step, for each
  * head whose max logit exceeds the threshold, rescale that head's query and

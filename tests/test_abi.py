@@ -64,6 +64,12 @@ def test_host_validation_without_gpu(lib):
     assert lib.mla_attn_fwd(G, 0, 1, 1, bad, ok, ok, ok, None, ok, ok, None) == -2
     assert lib.mla_attn_fwd(G, 7, 1, 1, ok, ok, ok, ok, None, ok, ok, None) == -1
     assert lib.mla_attn_fwd(G, 0, 1, 1, ok, ok, ok, ok, bad, ok, ok, None) == -2
+    # the fp32-output training form validates the same way
+    assert lib.mla_attn_fwd_train(None, 0, 1, 1, ok, ok, ok, ok, None, ok, ok, None) == -1
+    assert lib.mla_attn_fwd_train(G, 0, 1, 0, ok, ok, ok, ok, None, ok, ok, None) == -1
+    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, None, ok, None) == -1
+    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, bad, ok, None) == -2
+    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, ok, None, None) == -1
     # clip: tau must be positive and finite
     assert lib.qkclip_rescale(G, 0, ok, ok, ok, ctypes.c_float(0.0), None, None, None) == -1
     assert lib.qkclip_rescale(G, 0, ok, ok, ok, ctypes.c_float(float("inf")), None, None, None) == -1
