@@ -18,6 +18,8 @@ from .mla import (  # noqa: F401
     attention,
     attention_rows,
     head_maxlogit,
+    attention_lse,
+    attention_backward,
     qkclip,
     decode_absorbed,
     decode_materialised,

@@ -33,7 +33,7 @@ import numpy as np
 
 __all__ = [
     "bf16_round", "rms_norm", "up_proj", "attention", "attention_rows", "head_maxlogit",
-    "qkclip", "decode_absorbed", "decode_materialised", "layer_forward",
+    "attention_lse", "attention_backward", "qkclip", "decode_absorbed", "decode_materialised", "layer_forward",
 ]
 
 
@@ -224,6 +224,78 @@ def head_maxlogit(Q, KC, kS, heads, *, row_chunk=2048):
                 m_h = max(m_h, float(np.where(causal, S, -np.inf).max()))
         res[int(h)] = m_h
     return res
+
+
+# ---------------------------------------------------------------------------
+# Training: the row log-sum-exp the forward leaves for the backward, and the
+# gradients of the forward above.  The pages run this layer in training (the
+# clip exists for it: [SOTA] "Source"; [NOPE] "Un détail de précision
+# numérique" keeps the forward's output in FP32 while training); k^S being one
+# key part shared by every head ([OMA] "All 20 steps") makes its gradient a
+# sum over heads.
+# ---------------------------------------------------------------------------
+def attention_lse(Q, KC, kS):
+    """lse[b, t, h] = log sum_{s <= t} exp S_h[t, s], S the scaled logits."""
+    B, T, H, d_qk = Q.shape
+    scale = 1.0 / math.sqrt(d_qk)
+    out = np.empty((B, T, H))
+    causal = np.arange(T)[None, :] <= np.arange(T)[:, None]
+    for b in range(B):
+        for h in range(H):
+            K = _f64(_head_keys(KC, kS, b, h))
+            S = np.where(causal, (_f64(Q[b, :, h, :]) @ K.T) * scale, -np.inf)
+            m = S.max(axis=1, keepdims=True)
+            out[b, :, h] = (m + np.log(np.exp(S - m).sum(axis=1, keepdims=True)))[:, 0]
+    return out
+
+
+def attention_backward(Q, KC, kS, V, g, dO):
+    """Gradients of the loss through o = sigmoid(g) * causal-softmax(Q K^T/sqrt(d_qk)) V.
+
+    dO is dL/do [B, T, H*d_v].  Per batch item b and head h, with K_h =
+    [K^C_h | k^S], A the causal softmax and O~ = A V_h (chain rule, in order):
+      dO~     = dO * sigmoid(g)            dg = dO * O~ * sigmoid(g) (1 - sigmoid(g))
+      dV_h    = A^T dO~                    dA = dO~ V_h^T
+      dS      = A * (dA - rowsum(dA * A))  (softmax Jacobian; masked entries of A are 0)
+      dQ_h    = dS K_h / sqrt(d_qk)        dK_h = dS^T Q_h / sqrt(d_qk)
+    and dK_h splits into dK^C_h (its first d_c columns) and head h's share of
+    dk^S (the rest); dk^S is the sum of the shares over the heads.
+    Returns float64 (dQ [B,T,H,d_qk], dKC [B,T,H,d_c], dkS [B,T,d_s],
+    dV [B,T,H,d_v], dg [B,T,H*d_v] or None when g is None).
+    """
+    B, T, H, d_qk = Q.shape
+    d_c, d_v = KC.shape[-1], V.shape[-1]
+    scale = 1.0 / math.sqrt(d_qk)
+    dO = _f64(dO).reshape(B, T, H, d_v)
+    gg = None if g is None else _f64(g).reshape(B, T, H, d_v)
+    dQ = np.zeros((B, T, H, d_qk))
+    dKC = np.zeros((B, T, H, d_c))
+    dkS = np.zeros((B, T, d_qk - d_c))
+    dV = np.zeros((B, T, H, d_v))
+    dg = None if g is None else np.zeros((B, T, H, d_v))
+    causal = np.arange(T)[None, :] <= np.arange(T)[:, None]
+    for b in range(B):
+        for h in range(H):
+            K = _f64(_head_keys(KC, kS, b, h))
+            Qh, Vh = _f64(Q[b, :, h, :]), _f64(V[b, :, h, :])
+            S = np.where(causal, (Qh @ K.T) * scale, -np.inf)
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            A = P / P.sum(axis=1, keepdims=True)
+            Ot = A @ Vh
+            if gg is None:
+                dOt = dO[b, :, h, :]
+            else:
+                sg = _sigmoid(gg[b, :, h, :])
+                dOt = dO[b, :, h, :] * sg
+                dg[b, :, h, :] = dO[b, :, h, :] * Ot * sg * (1.0 - sg)
+            dV[b, :, h, :] = A.T @ dOt
+            dA = dOt @ Vh.T
+            dS = A * (dA - (dA * A).sum(axis=1, keepdims=True))
+            dQ[b, :, h, :] = (dS @ K) * scale
+            dK = (dS.T @ Qh) * scale
+            dKC[b, :, h, :] = dK[:, :d_c]
+            dkS[b] += dK[:, d_c:]
+    return dQ, dKC, dkS, dV, (None if dg is None else dg.reshape(B, T, H * d_v))
 
 
 # ---------------------------------------------------------------------------
