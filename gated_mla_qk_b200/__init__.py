@@ -7,6 +7,7 @@ its own kernels.  There is no CPU or library fallback: if the shared object is
 missing, importing the binding's functions raises.
 
 Entry points (same names as the C ABI): ``mla_up_proj``, ``mla_attn_fwd``, ``mla_attn_fwd_train``,
+``mla_attn_bwd``,
 ``qkclip_rescale``, ``mla_decode_absorbed``, ``mla_gemm``; plus the workspace
 size queries, ``device_status`` and ``launch_count``.
 """
@@ -24,7 +25,7 @@ GMLA_BF16, GMLA_F32 = 0, 1
 STATUS = {0: "GMLA_OK", -1: "GMLA_EINVAL", -2: "GMLA_EALIGN", -3: "GMLA_EUNSUPPORTED", -4: "GMLA_ECUDA",
           -5: "GMLA_ETIMEOUT", -6: "GMLA_EWORKSPACE"}
 
-EXPORTS = ["mla_up_proj_workspace", "mla_up_proj", "mla_attn_fwd", "mla_attn_fwd_train", "qkclip_rescale", "mla_decode_workspace",
+EXPORTS = ["mla_up_proj_workspace", "mla_up_proj", "mla_attn_fwd", "mla_attn_fwd_train", "mla_attn_bwd_workspace", "mla_attn_bwd", "qkclip_rescale", "mla_decode_workspace",
            "mla_decode_absorbed", "mla_decode_absorbed_noalloc", "mla_gemm", "gmla_device_status", "gmla_last_cuda_error", "gmla_strerror",
            "gmla_version", "gmla_launch_count"]
 
@@ -67,7 +68,9 @@ def load_library(path: str = LIB_PATH):
         "mla_up_proj_workspace": (S, [G, I, I, I]),
         "mla_up_proj": (I, [G, I, I, I] + [P] * 12 + [P, S, P]),
         "mla_attn_fwd": (I, [G, I, I, I, P, P, P, P, P, P, P, P]),
-        "mla_attn_fwd_train": (I, [G, I, I, I, P, P, P, P, P, P, P, P]),
+        "mla_attn_fwd_train": (I, [G, I, I, I, P, P, P, P, P, P, P, P, P]),
+        "mla_attn_bwd_workspace": (S, [G, I, I]),
+        "mla_attn_bwd": (I, [G, I, I, I] + [P] * 13 + [P, S, P]),
         "qkclip_rescale": (I, [G, I, P, P, P, F, P, P, P]),
         "mla_decode_workspace": (S, [G, I, I, I]),
         "mla_decode_absorbed": (I, [G, I, I, P, P, P, P, I, P, P, P, S, P]),
@@ -162,16 +165,36 @@ def mla_attn_fwd(geom: Geom, Q, KC, kS, V, g, O, maxlogit, stream=None):
         _stream(stream)))
 
 
-def mla_attn_fwd_train(geom: Geom, Q, KC, kS, V, g, O, maxlogit, stream=None):
-    """mla_attn_fwd with the output O kept in float32 (the training form)."""
+def mla_attn_fwd_train(geom: Geom, Q, KC, kS, V, g, O, maxlogit, lse=None, stream=None):
+    """mla_attn_fwd with the output O kept in float32 (the training form); lse (optional) gets the row log-sum-exp."""
     lib = load_library()
     torch = _torch()
     B, T = Q.shape[0], Q.shape[1]
     dt = _dtype_code(Q)
     _check("mla_attn_fwd_train", lib.mla_attn_fwd_train(
         ctypes.byref(CGeom.of(geom)), dt, B, T, _ptr(Q, "Q"), _ptr(KC, "KC", Q.dtype), _ptr(kS, "kS", Q.dtype),
-        _ptr(V, "V", Q.dtype), _ptr(g, "g", Q.dtype), _ptr(O, "O", torch.float32),
+        _ptr(V, "V", Q.dtype), _ptr(g, "g", Q.dtype), _ptr(O, "O", torch.float32), _ptr(lse, "lse", torch.float32),
         _ptr(maxlogit, "maxlogit", torch.float32), _stream(stream)))
+
+
+def mla_attn_bwd_workspace(geom: Geom, B: int, T: int) -> int:
+    return load_library().mla_attn_bwd_workspace(ctypes.byref(CGeom.of(geom)), B, T)
+
+
+def mla_attn_bwd(geom: Geom, Q, KC, kS, V, g, O, lse, dO, dQ, dKC, dkS, dV, dg=None, workspace=None, stream=None):
+    """Gradients (float32) of the loss through the gated attention: dQ, dKC, dkS (summed over heads), dV, dg."""
+    lib = load_library()
+    torch = _torch()
+    B, T = Q.shape[0], Q.shape[1]
+    f32 = torch.float32
+    if workspace is None:
+        workspace = torch.empty(mla_attn_bwd_workspace(geom, B, T), dtype=torch.uint8, device=Q.device)
+    _check("mla_attn_bwd", lib.mla_attn_bwd(
+        ctypes.byref(CGeom.of(geom)), _dtype_code(Q), B, T, _ptr(Q, "Q"), _ptr(KC, "KC", Q.dtype),
+        _ptr(kS, "kS", Q.dtype), _ptr(V, "V", Q.dtype), _ptr(g, "g", Q.dtype), _ptr(O, "O", f32),
+        _ptr(lse, "lse", f32), _ptr(dO, "dO", f32), _ptr(dQ, "dQ", f32), _ptr(dKC, "dKC", f32),
+        _ptr(dkS, "dkS", f32), _ptr(dV, "dV", f32), _ptr(dg, "dg", f32), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def qkclip_rescale(geom: Geom, W_UQ, W_UKV, maxlogit, tau: float, clipped=None, gamma=None, stream=None):

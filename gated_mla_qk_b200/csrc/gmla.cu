@@ -16,6 +16,7 @@
 #include "tc_attn.cuh"
 #include "tc_decode.cuh"
 #include "tc_gemm.cuh"
+#include "attn_bwd.cuh"
 
 namespace gmla {
 
@@ -178,7 +179,8 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
 // Attention forward dispatch
 // ---------------------------------------------------------------------------
 static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const void* KC, const void* kS,
-                       const void* V, const void* gate, void* O, bool out_f32, float* maxlogit, cudaStream_t st) {
+                       const void* V, const void* gate, void* O, bool out_f32, float* maxlogit, float* lse,
+                       cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -200,6 +202,7 @@ static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const vo
   p.g = static_cast<const __nv_bfloat16*>(gate);
   p.O = O;
   p.maxlogit = maxlogit;
+  p.lse = lse;
   p.scale = 1.f / std::sqrt(192.f);
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   simt::fill_kernel<<<(H + 127) / 128, 128, 0, st>>>(maxlogit, H, -INFINITY);
@@ -391,7 +394,7 @@ int mla_attn_fwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void*
   cudaStream_t st = as_stream(stream);
   if (dtype == GMLA_BF16 && is_k3_head_geometry(g)) {
     if ((long long)B * T * g->H * 192 >= (1LL << 40)) return GMLA_EUNSUPPORTED;
-    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, false, maxlogit, st);
+    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, false, maxlogit, nullptr, st);
   }
   if (g->d_c + g->d_s > 256 || g->d_v > simt::kAttnMaxDV) return GMLA_EUNSUPPORTED;
   if (dtype == GMLA_F32)
@@ -405,25 +408,59 @@ int mla_attn_fwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void*
 // ---------------------------------------------------------------------------
 // Training variant: the same forward with o kept in fp32.
 int mla_attn_fwd_train(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void* Q, const void* KC,
-                       const void* kS, const void* V, const void* gate, float* O, float* maxlogit, void* stream) {
+                       const void* kS, const void* V, const void* gate, float* O, float* lse, float* maxlogit,
+                       void* stream) {
   GMLA_TRY(check_geom(g));
   GMLA_TRY(check_dtype(dtype));
   if (B <= 0 || T <= 0) return GMLA_EINVAL;
   GMLA_REQUIRE(Q); GMLA_REQUIRE(KC); GMLA_REQUIRE(V); GMLA_REQUIRE(O); GMLA_REQUIRE(maxlogit);
   if (g->d_s > 0) GMLA_REQUIRE(kS);
   GMLA_OPTIONAL(gate);
+  GMLA_OPTIONAL(lse);
   cudaStream_t st = as_stream(stream);
   if (dtype == GMLA_BF16 && is_k3_head_geometry(g)) {
     if ((long long)B * T * g->H * 192 >= (1LL << 40)) return GMLA_EUNSUPPORTED;
-    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, true, maxlogit, st);
+    return attn_fwd_tc(g, B, T, Q, KC, kS, V, gate, O, true, maxlogit, lse, st);
   }
   if (g->d_c + g->d_s > 256 || g->d_v > simt::kAttnMaxDV) return GMLA_EUNSUPPORTED;
   if (dtype == GMLA_F32)
     return simt::attn_fwd<float>(B, T, g->H, g->d_c, g->d_s, g->d_v, (const float*)Q, (const float*)KC,
-                                 (const float*)kS, (const float*)V, (const float*)gate, O, maxlogit, st);
+                                 (const float*)kS, (const float*)V, (const float*)gate, O, maxlogit, st, lse);
   using bf = __nv_bfloat16;
   return simt::attn_fwd<bf, float>(B, T, g->H, g->d_c, g->d_s, g->d_v, (const bf*)Q, (const bf*)KC, (const bf*)kS,
-                                   (const bf*)V, (const bf*)gate, O, maxlogit, st);
+                                   (const bf*)V, (const bf*)gate, O, maxlogit, st, lse);
+}
+
+// ---------------------------------------------------------------------------
+// Backward of the training forward.
+size_t mla_attn_bwd_workspace(const gmla_geom* g, int B, int T) {
+  if (check_geom(g) != GMLA_OK || B <= 0 || T <= 0) return 0;
+  return bwd::workspace_bytes(B, T, g->H, g->d_v);
+}
+
+int mla_attn_bwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void* Q, const void* KC, const void* kS,
+                 const void* V, const void* gate, const float* O, const float* lse, const float* dO, float* dQ,
+                 float* dKC, float* dkS, float* dV, float* dg, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  if (B <= 0 || T <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(Q); GMLA_REQUIRE(KC); GMLA_REQUIRE(V); GMLA_REQUIRE(O); GMLA_REQUIRE(lse); GMLA_REQUIRE(dO);
+  GMLA_REQUIRE(dQ); GMLA_REQUIRE(dKC); GMLA_REQUIRE(dV);
+  if (g->d_s > 0) { GMLA_REQUIRE(kS); GMLA_REQUIRE(dkS); }
+  GMLA_OPTIONAL(gate);
+  if (gate) GMLA_REQUIRE(dg);
+  if (g->d_c + g->d_s > bwd::kMaxD || g->d_v > bwd::kMaxD) return GMLA_EUNSUPPORTED;
+  if (!workspace || workspace_bytes < bwd::workspace_bytes(B, T, g->H, g->d_v)) return GMLA_EWORKSPACE;
+  if (!aligned16(workspace)) return GMLA_EALIGN;
+  cudaStream_t st = as_stream(stream);
+  bwd::Dims p{B, T, g->H, g->d_c, g->d_s, g->d_v, 1.f / std::sqrt((float)(g->d_c + g->d_s))};
+  if (dtype == GMLA_F32)
+    return bwd::run<float>(p, (const float*)Q, (const float*)KC, (const float*)kS, (const float*)V,
+                           (const float*)gate, O, lse, dO, dQ, dKC, dkS, dV, dg, workspace, st);
+  using bf = __nv_bfloat16;
+  return bwd::run<bf>(p, (const bf*)Q, (const bf*)KC, (const bf*)kS, (const bf*)V, (const bf*)gate, O, lse, dO, dQ,
+                      dKC, dkS, dV, dg, workspace, st);
 }
 
 // ---------------------------------------------------------------------------

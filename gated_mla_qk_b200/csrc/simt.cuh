@@ -148,7 +148,7 @@ template <typename T, typename TO = T>
 __global__ void __launch_bounds__(128) attn_fwd_kernel(
     int T_, int H, int d_c, int d_s, int d_v, const T* __restrict__ Q, const T* __restrict__ KC,
     const T* __restrict__ kS, const T* __restrict__ V, const T* __restrict__ g, TO* __restrict__ O,
-    float* __restrict__ maxlogit, float scale) {
+    float* __restrict__ maxlogit, float* __restrict__ lse, float scale) {
   extern __shared__ float smem[];
   const int d_qk = d_c + d_s;
   float* sQ = smem;                               // [BQ][d_qk]
@@ -223,6 +223,7 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(
   }
   // Output row and the head's max logit (m_run is the exact row max here).
   if (t_row < T_) {
+    if (lse && lane8 == 0) lse[((size_t)b * T_ + t_row) * H + h] = m_run + logf(l_run);
     const float inv_l = 1.f / l_run;
     for (int k = 0; k < n_cols; ++k) {
       const int c = lane8 + 8 * k;
@@ -252,7 +253,7 @@ inline size_t attn_smem_bytes(int d_qk, int d_v) {
 
 template <typename T, typename TO = T>
 inline int attn_fwd(int B, int T_, int H, int d_c, int d_s, int d_v, const T* Q, const T* KC, const T* kS,
-                    const T* V, const T* g, TO* O, float* maxlogit, cudaStream_t st) {
+                    const T* V, const T* g, TO* O, float* maxlogit, cudaStream_t st, float* lse = nullptr) {
   const size_t smem = attn_smem_bytes(d_c + d_s, d_v);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<T, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -260,7 +261,7 @@ inline int attn_fwd(int B, int T_, int H, int d_c, int d_s, int d_v, const T* Q,
   }
   fill_kernel<<<(H + 127) / 128, 128, 0, st>>>(maxlogit, H, -INFINITY);
   dim3 grid((T_ + kAttnBQ - 1) / kAttnBQ, H, B);
-  attn_fwd_kernel<T, TO><<<grid, 128, smem, st>>>(T_, H, d_c, d_s, d_v, Q, KC, kS, V, g, O, maxlogit,
+  attn_fwd_kernel<T, TO><<<grid, 128, smem, st>>>(T_, H, d_c, d_s, d_v, Q, KC, kS, V, g, O, maxlogit, lse,
                                               1.f / sqrtf((float)(d_c + d_s)));
   note_launches(2);
   return check_launch();

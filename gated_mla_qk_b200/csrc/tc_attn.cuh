@@ -53,6 +53,7 @@ struct Params {
   const __nv_bfloat16* g;   // [B][T][H*128] or nullptr
   void* O;                  // [B][T][H*128], bf16 or (training variant) fp32
   float* maxlogit;          // [H]
+  float* lse;               // [B][T][H] row log-sum-exp of the scaled logits, or nullptr
   float scale;              // 1/sqrt(192)
   float scale_log2;         // log2(e)/sqrt(192)
 };
@@ -325,6 +326,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
+      if (p.lse && valid) p.lse[((size_t)b * p.T + t) * p.H + h] = fmaf(m_used, p.scale, __logf(l));
       float v = valid ? true_max * p.scale : -INFINITY;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

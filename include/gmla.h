@@ -110,14 +110,43 @@ int mla_attn_fwd(const gmla_geom* geom, gmla_dtype dtype, int B, int T,
  * (the attention output stays in FP32 during training, so no biased
  * rounding of o to bf16).  Arguments, layouts, ownership and errors are those
  * of mla_attn_fwd except:
- *   O [B][T][H*d_v] float32 (written) whatever `dtype` is.
+ *   O [B][T][H*d_v] float32 (written) whatever `dtype` is;
+ *   lse (nullable) [B][T][H] float32 (written): log sum_{s<=t} exp S_h[t][s]
+ *     of the scaled logits, the row statistic mla_attn_bwd recomputes A from.
  * bf16 with d_c=128, d_s=64, d_v=128 runs the tcgen05/TMA kernel (its epilogue
  * stores from registers: no output tile is staged in shared memory); other
  * shapes and fp32 inputs run the CUDA-core kernel with fp32 output.
  */
 int mla_attn_fwd_train(const gmla_geom* geom, gmla_dtype dtype, int B, int T,
                        const void* Q, const void* KC, const void* kS, const void* V,
-                       const void* g, float* O, float* maxlogit, void* stream);
+                       const void* g, float* O, float* lse, float* maxlogit, void* stream);
+
+/* Bytes of scratch mla_attn_bwd needs (0 for a bad geometry or size). */
+size_t mla_attn_bwd_workspace(const gmla_geom* geom, int B, int T);
+
+/*
+ * mla_attn_bwd — gradients of a loss L through the forward above (the layer
+ * is trained: "Anthology of the SOTA" SOTA-131 "Source" clips it during
+ * training; "Gated MLA et NoPE", "Un détail de précision numérique").  With
+ * the forward of mla_attn_fwd ("Kimi K3 · Gated MLA · OpenModelAtlas",
+ * "All 20 steps") and A_ts = exp(S_ts - lse_t) for s <= t:
+ *   dO~ = dO * sigmoid(g);  dg = dO * o * (1 - sigmoid(g));  D_t = sum_c dO * o
+ *   dS = A * (dO~ V_h^T - D);  dQ_h = dS K_h / sqrt(d_qk);  dV_h = A^T dO~
+ *   dK_h = dS^T Q_h / sqrt(d_qk) -> dKC (first d_c columns), and dkS = the
+ *   sum over heads of the last d_s columns (k^S is shared by every head).
+ * Inputs: Q, KC, kS, V, g as for mla_attn_fwd, in `dtype`; O (= o) and lse
+ *   from mla_attn_fwd_train; dO = dL/do [B][T][H*d_v] float32.
+ * Outputs (written, not accumulated), float32 in the layouts of the inputs:
+ *   dQ [B][T][H][d_c+d_s], dKC [B][T][H][d_c], dkS [B][T][d_s],
+ *   dV [B][T][H][d_v], dg [B][T][H*d_v] (required when g is given).
+ * workspace: device scratch of at least mla_attn_bwd_workspace() bytes.
+ * CUDA-core kernels, fp32 arithmetic; d_c+d_s <= 256, d_v <= 256.
+ */
+int mla_attn_bwd(const gmla_geom* geom, gmla_dtype dtype, int B, int T,
+                 const void* Q, const void* KC, const void* kS, const void* V, const void* g,
+                 const float* O, const float* lse, const float* dO,
+                 float* dQ, float* dKC, float* dkS, float* dV, float* dg,
+                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * qkclip_rescale — QK-Clip applied to the weights, in place.

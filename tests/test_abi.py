@@ -64,12 +64,24 @@ def test_host_validation_without_gpu(lib):
     assert lib.mla_attn_fwd(G, 0, 1, 1, bad, ok, ok, ok, None, ok, ok, None) == -2
     assert lib.mla_attn_fwd(G, 7, 1, 1, ok, ok, ok, ok, None, ok, ok, None) == -1
     assert lib.mla_attn_fwd(G, 0, 1, 1, ok, ok, ok, ok, bad, ok, ok, None) == -2
-    # the fp32-output training form validates the same way
-    assert lib.mla_attn_fwd_train(None, 0, 1, 1, ok, ok, ok, ok, None, ok, ok, None) == -1
-    assert lib.mla_attn_fwd_train(G, 0, 1, 0, ok, ok, ok, ok, None, ok, ok, None) == -1
-    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, None, ok, None) == -1
-    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, bad, ok, None) == -2
-    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, ok, None, None) == -1
+    # the fp32-output training form validates the same way (lse is optional)
+    assert lib.mla_attn_fwd_train(None, 0, 1, 1, ok, ok, ok, ok, None, ok, None, ok, None) == -1
+    assert lib.mla_attn_fwd_train(G, 0, 1, 0, ok, ok, ok, ok, None, ok, None, ok, None) == -1
+    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, None, None, ok, None) == -1
+    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, bad, None, ok, None) == -2
+    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, ok, bad, ok, None) == -2
+    assert lib.mla_attn_fwd_train(G, 0, 1, 1, ok, ok, ok, ok, None, ok, None, None, None) == -1
+    # backward: every gradient buffer, O, lse, dO and a large enough workspace are required
+    bneed = lib.mla_attn_bwd_workspace(G, 1, 1)
+    assert bneed > 0 and lib.mla_attn_bwd_workspace(None, 1, 1) == 0
+    full = lambda **kw: [kw.get(n, ok) for n in ("Q", "KC", "kS", "V", "g", "O", "lse", "dO", "dQ", "dKC", "dkS", "dV", "dg")]
+    assert lib.mla_attn_bwd(G, 0, 0, 1, *full(), ok, bneed, None) == -1
+    assert lib.mla_attn_bwd(G, 0, 1, 1, *full(lse=None), ok, bneed, None) == -1
+    assert lib.mla_attn_bwd(G, 0, 1, 1, *full(dkS=None), ok, bneed, None) == -1
+    assert lib.mla_attn_bwd(G, 0, 1, 1, *full(dg=None), ok, bneed, None) == -1        # gated needs dg
+    assert lib.mla_attn_bwd(G, 0, 1, 1, *full(dQ=bad), ok, bneed, None) == -2
+    assert lib.mla_attn_bwd(G, 0, 1, 1, *full(), ok, bneed - 1, None) == -6
+    assert lib.mla_attn_bwd(G, 0, 1, 1, *full(), None, bneed, None) == -6
     # clip: tau must be positive and finite
     assert lib.qkclip_rescale(G, 0, ok, ok, ok, ctypes.c_float(0.0), None, None, None) == -1
     assert lib.qkclip_rescale(G, 0, ok, ok, ok, ctypes.c_float(float("inf")), None, None, None) == -1

@@ -1,0 +1,66 @@
+"""Parity of the training forward's log-sum-exp and of mla_attn_bwd with the
+oracle (whose backward is pinned by finite differences and torch autograd)."""
+import numpy as np
+import pytest
+
+import oracle
+from gated_mla_qk_b200 import synth
+from gpu_util import TOL_BF16, check_status, dev, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _train_and_backward(inp, geom, dO, gate):
+    import torch
+    import gated_mla_qk_b200 as gm
+    B, T = inp["Q"].shape[:2]
+    H = geom.H
+    Q, KC, kS, V = (dev(inp[k], "bf16") for k in ("Q", "KC", "kS", "V"))
+    g = dev(inp["g"], "bf16") if gate else None
+    f32 = dict(dtype=torch.float32, device="cuda")
+    O = torch.empty(B, T, H * geom.d_v, **f32)
+    lse = torch.empty(B, T, H, **f32)
+    ml = torch.empty(H, **f32)
+    gm.mla_attn_fwd_train(geom, Q, KC, kS, V, g, O, ml, lse=lse)
+    dQ = torch.empty(B, T, H, geom.d_qk, **f32)
+    dKC = torch.empty(B, T, H, geom.d_c, **f32)
+    dkS = torch.empty(B, T, geom.d_s, **f32)
+    dV = torch.empty(B, T, H, geom.d_v, **f32)
+    dg = torch.empty(B, T, H * geom.d_v, **f32) if gate else None
+    gm.mla_attn_bwd(geom, Q, KC, kS, V, g, O, lse, torch.from_numpy(dO).cuda(), dQ, dKC, dkS, dV, dg)
+    check_status()
+    return host(lse), [host(x) if x is not None else None for x in (dQ, dKC, dkS, dV, dg)]
+
+
+@pytest.mark.parametrize("B,T,H,gate", [(1, 1, 2, True), (1, 70, 2, True), (2, 129, 3, False), (1, 300, 2, True)])
+def test_backward_k3_heads(B, T, H, gate):
+    """K3 head widths (the tcgen05 training forward feeds o and lse)."""
+    geom = synth.Geom(H=H)
+    inp = synth.attn_core(B, T, geom, seed=300 + T, hot_heads=1, hot_scale=3.0, gate=gate)
+    dO = np.random.default_rng(301 + T).standard_normal((B, T, H * geom.d_v)).astype(np.float32)
+    lse, got = _train_and_backward(inp, geom, dO, gate)
+    assert np.allclose(lse, oracle.attention_lse(inp["Q"], inp["KC"], inp["kS"]), rtol=1e-5, atol=1e-5)
+    want = oracle.attention_backward(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"] if gate else None, dO)
+    scale = np.linalg.norm(want[3])                  # dV: never zero
+    for name, a, b in zip(("dQ", "dKC", "dkS", "dV", "dg"), got, want):
+        if b is None:
+            assert a is None
+            continue
+        a = a.reshape(b.shape)
+        if np.linalg.norm(b) == 0:                    # T = 1: one key, so dS = 0 exactly
+            assert np.linalg.norm(a) <= 1e-4 * scale, name
+            continue
+        # o comes from the bf16 tensor-core forward (P rounded to bf16), which D = sum dO * o inherits
+        assert rel_l2(a, b) <= TOL_BF16, name
+
+
+def test_backward_other_head_widths_fp32_path():
+    """Other head widths: CUDA-core forward and backward, all fp32 arithmetic."""
+    geom = synth.TINY
+    inp = synth.attn_core(1, 45, geom, seed=311, hot_heads=1, hot_scale=2.0, gate=True)
+    dO = np.random.default_rng(312).standard_normal((1, 45, geom.H * geom.d_v)).astype(np.float32)
+    lse, got = _train_and_backward(inp, geom, dO, True)
+    assert np.allclose(lse, oracle.attention_lse(inp["Q"], inp["KC"], inp["kS"]), rtol=1e-5, atol=1e-5)
+    want = oracle.attention_backward(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"], dO)
+    for name, a, b in zip(("dQ", "dKC", "dkS", "dV", "dg"), got, want):
+        assert rel_l2(a.reshape(b.shape), b) <= 1e-4, name
