@@ -40,6 +40,65 @@ B_FWD, T_FWD = 1, 16384
 FWD_FLOP = 2.0 * B_FWD * 96 * T_FWD * (T_FWD + 1) / 2 * (192 + 128)
 
 
+T_TRAIN = 4096
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # CUDA-core fp32 FMA peak at the maximum SM clock
+
+
+def train_leg(args, gm, synth, geom, rank, st, dist):
+    """mla_attn_fwd_train + mla_attn_bwd at B=1, T=4096, H=96 (gated, K3 heads)."""
+    import torch
+    tin = synth.attn_core(1, T_TRAIN, geom, seed=5 + 1000 * rank, hot_heads=8, hot_scale=4.0)
+    td = {k: synth.to_torch(v, "bf16", "cuda") for k, v in tin.items()}
+    del tin
+    H, T = geom.H, T_TRAIN
+    f32 = dict(dtype=torch.float32, device="cuda")
+    O = torch.empty(1, T, H * 128, **f32)
+    lse = torch.empty(1, T, H, **f32)
+    ml = torch.empty(H, **f32)
+    gen = torch.Generator(device="cuda").manual_seed(6 + rank)
+    dO = torch.randn(1, T, H * 128, generator=gen, **f32)
+    dQ = torch.empty(1, T, H, 192, **f32)
+    dKC = torch.empty(1, T, H, 128, **f32)
+    dkS = torch.empty(1, T, 64, **f32)
+    dV = torch.empty(1, T, H, 128, **f32)
+    dg = torch.empty(1, T, H * 128, **f32)
+    ws = torch.empty(gm.mla_attn_bwd_workspace(geom, 1, T), dtype=torch.uint8, device="cuda")
+
+    def run(ev):
+        ev[0].record(st)
+        gm.mla_attn_fwd_train(geom, td["Q"], td["KC"], td["kS"], td["V"], td["g"], O, ml, lse=lse)
+        ev[1].record(st)
+        gm.mla_attn_bwd(geom, td["Q"], td["KC"], td["kS"], td["V"], td["g"], O, lse, dO, dQ, dKC, dkS, dV, dg, ws)
+        ev[2].record(st)
+
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(args.warmup):
+        run(warm)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        run(evs[k])
+    torch.cuda.synchronize()
+    t = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps,
+                      sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    f_ms, b_ms = t.tolist()
+    pairs = H * T * (T + 1) / 2
+    f_flop = 2.0 * pairs * (192 + 128)
+    b_flop = 2.0 * pairs * (2 * 128 + 2 * 192)          # dV, dA, dQ, dK products (recomputation not counted)
+    return {
+        "attn_fwd_train_B1_T4096": {"ms": f_ms, "value": f_flop / (f_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                                    "what": "mla_attn_fwd_train (fp32 o, lse)"},
+        "attn_bwd_B1_T4096": {"ms": b_ms, "value": b_flop / (b_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                              "what": "mla_attn_bwd, CUDA-core fp32",
+                              "roofline": {"bound": "alu", "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                                           "frac": b_flop / (b_ms / 1e3) / 1e12 / FP32_PEAK_TFLOPS}},
+    }
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -52,6 +111,7 @@ def parse():
     ap.add_argument("--skip-decode", action="store_true", help="time the forward alone (profiling runs)")
     ap.add_argument("--skip-fwd", action="store_true", help="time the decode alone (profiling runs)")
     ap.add_argument("--skip-clip", action="store_true", help="leave out the K3 QK-Clip chain (profiling runs)")
+    ap.add_argument("--no-train", action="store_true", help="skip the training-form leg (fp32-output forward + backward)")
     return ap.parse_args()
 
 
@@ -376,6 +436,11 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms.item(),
                "what": "mla_attn_fwd with inputs copied from pinned host memory and O + maxlogit copied back"}
 
+    # ---- training form, timed on its own after the step: fp32-output forward + backward ----
+    train = None
+    if not args.no_train:
+        train = train_leg(args, gm, synth, geom, rank, st, dist)
+
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -440,6 +505,8 @@ def main():
         }
     line["parts"]["attn_fwd_B1_T16384"] = {"ms": fwd_avg_ms, "value": fwd_tflops, "unit": "TFLOP/s"}
     line["parts"]["decode_64seq"] = {"ms": dec_avg_ms, "value": dec_gbs, "unit": "GB/s"}
+    if train:
+        line["parts"].update(train)
     if e2e:
         line["e2e"] = e2e
     if not args.no_cpu_baseline and T_run == T_FWD:
