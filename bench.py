@@ -41,7 +41,6 @@ FWD_FLOP = 2.0 * B_FWD * 96 * T_FWD * (T_FWD + 1) / 2 * (192 + 128)
 
 
 T_TRAIN = 4096
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # CUDA-core fp32 FMA peak at the maximum SM clock
 
 
 def train_leg(args, gm, synth, geom, rank, st, dist):
@@ -87,15 +86,16 @@ def train_leg(args, gm, synth, geom, rank, st, dist):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     f_ms, b_ms = t.tolist()
     pairs = H * T * (T + 1) / 2
+    pk_bf16 = peaks()["bf16"]
     f_flop = 2.0 * pairs * (192 + 128)
     b_flop = 2.0 * pairs * (2 * 128 + 2 * 192)          # dV, dA, dQ, dK products (recomputation not counted)
     return {
         "attn_fwd_train_B1_T4096": {"ms": f_ms, "value": f_flop / (f_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                                     "what": "mla_attn_fwd_train (fp32 o, lse)"},
         "attn_bwd_B1_T4096": {"ms": b_ms, "value": b_flop / (b_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-                              "what": "mla_attn_bwd, CUDA-core fp32",
-                              "roofline": {"bound": "alu", "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                                           "frac": b_flop / (b_ms / 1e3) / 1e12 / FP32_PEAK_TFLOPS}},
+                              "what": "mla_attn_bwd, warp-level bf16 tensor-core passes (mma.sync), fp32 accumulation",
+                              "roofline": {"bound": "tensor", "peak": pk_bf16, "unit": "TFLOP/s",
+                                           "frac": b_flop / (b_ms / 1e3) / 1e12 / pk_bf16}},
     }
 
 

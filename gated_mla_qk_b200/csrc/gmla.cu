@@ -459,6 +459,9 @@ int mla_attn_bwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void*
     return bwd::run<float>(p, (const float*)Q, (const float*)KC, (const float*)kS, (const float*)V,
                            (const float*)gate, O, lse, dO, dQ, dKC, dkS, dV, dg, workspace, st);
   using bf = __nv_bfloat16;
+  if (is_k3_head_geometry(g))
+    return bwd::run_tc(p, (const bf*)Q, (const bf*)KC, (const bf*)kS, (const bf*)V, (const bf*)gate, O, lse, dO, dQ,
+                       dKC, dkS, dV, dg, workspace, st);
   return bwd::run<bf>(p, (const bf*)Q, (const bf*)KC, (const bf*)kS, (const bf*)V, (const bf*)gate, O, lse, dO, dQ,
                       dKC, dkS, dV, dg, workspace, st);
 }

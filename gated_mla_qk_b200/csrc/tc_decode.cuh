@@ -434,29 +434,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   }
 }
 
-// ---------------------------------------------------------------------------
-// Warp-level bf16 MMA (m16n8k16, fp32 accumulate) for the two small products
-// around the split kernel: the absorbed query and the W_UV projection.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
-__device__ __forceinline__ uint32_t pack2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
-  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
-}
-
-__device__ __forceinline__ uint32_t lds32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t& r0, uint32_t& r1, const __nv_bfloat16* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r0), "=r"(r1) : "r"(smem_u32(p)));
-}
-
 // Work plan of the split kernel, built by one block of 256 threads:
-//   plan[0..n]        P_i = number of 64-token tiles of sequences 0..i-1
+//   plan[0..n]        P_i = number of BT-token tiles of sequences 0..i-1
 //   plan[n+1+c]       the sequence holding tile floor(c P_n / G), c < G
 __device__ void build_plan(int n_seq, const int* __restrict__ offs, int G, int* __restrict__ plan) {
   __shared__ int wsum[8];

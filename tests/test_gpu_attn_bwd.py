@@ -48,7 +48,8 @@ def test_backward_k3_heads(B, T, H, gate):
             continue
         a = a.reshape(b.shape)
         if np.linalg.norm(b) == 0:                    # T = 1: one key, so dS = 0 exactly
-            assert np.linalg.norm(a) <= 1e-4 * scale, name
+            # (the tensor-core passes take dO~ in bf16 for dA, D in fp32: bf16-level residue)
+            assert np.linalg.norm(a) <= TOL_BF16 * scale, name
             continue
         # o comes from the bf16 tensor-core forward (P rounded to bf16), which D = sum dO * o inherits
         assert rel_l2(a, b) <= TOL_BF16, name
