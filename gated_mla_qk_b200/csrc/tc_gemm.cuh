@@ -26,7 +26,10 @@ constexpr uint32_t A_BYTES = BM * BK * 2;                 // 16 KB
 constexpr uint32_t BSUB = BK * 128;                       // one 64 (k) x 64 (n) sub-tile, 8 KB
 constexpr uint32_t B_BYTES = 4 * BSUB;                    // 32 KB
 constexpr uint32_t STAGE = A_BYTES + B_BYTES;             // 48 KB
-constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
+constexpr uint32_t OFF_EPI = NSTAGE * STAGE;             // epilogue staging: 4 warps x [32 rows][64 cols + 8] bf16
+constexpr int EPI_LD = 72;                                // padded row (144 B): conflict-free 16-byte stores
+constexpr uint32_t EPI_WARP = 32 * EPI_LD * 2;            // 4.5 KB
+constexpr uint32_t OFF_BAR = OFF_EPI + 4 * EPI_WARP;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
 
 enum Bar { FULL = 0, EMPTY = NSTAGE, ACCF = 2 * NSTAGE, ACCE = ACCF + 2, DRAIN = ACCE + 2, NBAR = DRAIN + 1 };
@@ -125,32 +128,44 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
       const int tn = tile % n_tiles_n, tm = tile / n_tiles_n;
-      const int row = tm * BM + sub * 32 + lane;
       const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + 256u * (uint32_t)acc;
+      // 64 columns at a time: thread `lane` stages row 32*sub + lane of the
+      // chunk, then the warp writes the chunk out row by row, 8 lanes per
+      // row (a full 128-byte line), 4 rows per store instruction.
+      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem_raw + (sbase - sraw) + OFF_EPI + sub * EPI_WARP);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(taddr + 32u * c, v);
-        tmem_wait_ld_dep(v);
-        const int col0 = tn * BN + 32 * c;
-        if (row < p.M && col0 < p.N) {
+      for (int q = 0; q < BN / 64; ++q) {
+        float v[64];
+        tmem_ld32(taddr + 64u * q, *reinterpret_cast<float(*)[32]>(&v[0]));
+        tmem_ld32(taddr + 64u * q + 32u, *reinterpret_cast<float(*)[32]>(&v[32]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&v[0]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&v[32]));
+        __syncwarp();
+        uint4* srow = reinterpret_cast<uint4*>(stg + lane * EPI_LD);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          srow[c] = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                               pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+        __syncwarp();
+        const int col = tn * BN + 64 * q + 8 * (lane & 7);      // this lane's 8 columns
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          const int row = tm * BM + sub * 32 + r;
+          if (row >= p.M || col >= p.N) continue;
+          const uint4 val = reinterpret_cast<const uint4*>(stg + r * EPI_LD)[lane & 7];
           __nv_bfloat16* dst;
           if (p.mode == 1) {
-            const int h = col0 / 256, jj = col0 % 256;
+            const int h = col / 256, jj = col % 256;
             dst = (jj < 128) ? p.KC + ((size_t)row * p.H + h) * 128 + jj : p.V + ((size_t)row * p.H + h) * 128 + (jj - 128);
           } else {
-            dst = p.C + (size_t)row * p.N + col0;
+            dst = p.C + (size_t)row * p.N + col;
           }
-          if (col0 + 32 <= p.N) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              d4[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                 pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          if (col + 8 <= p.N) {
+            *reinterpret_cast<uint4*>(dst) = val;
           } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (col0 + e < p.N) dst[e] = __float2bfloat16_rn(v[e]);
+            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&val);
+            for (int k = 0; col + k < p.N; ++k) dst[k] = e[k];
           }
         }
       }
