@@ -105,6 +105,25 @@ static int make_map_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d
   return r == CUDA_SUCCESS ? GMLA_OK : GMLA_EUNSUPPORTED;
 }
 
+// Launch `k` on `st` with programmatic stream serialisation: the grid may be
+// scheduled before the previous kernel on the stream has finished, and must
+// call griddep_wait() before it reads anything that kernel writes.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_after_prev(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 static bool is_k3_head_geometry(const gmla_geom* g) { return g->d_c == 128 && g->d_s == 64 && g->d_v == 128; }
 
 // The tensor-core decode is specialised for Kimi K3's heads and latent.
@@ -126,8 +145,8 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
     attr_err = cudaFuncSetAttribute(tc_dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)tc_dec::SMEM_BYTES);
     if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(tc_dec::project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)tc_dec::PRJ_SMEM);
+      attr_err = cudaFuncSetAttribute(tc_dec::merge_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tc_dec::MP_SMEM);
     if (attr_err == cudaSuccess)
       attr_err = cudaFuncSetAttribute(tc_dec::absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)tc_dec::ABS_SMEM);
@@ -150,8 +169,6 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   float* part_ml = reinterpret_cast<float*>(p);
   p += al(np * tc_dec::HEADS * 2 * 4);
   float* part_u = reinterpret_cast<float*>(p);
-  p += al(np * tc_dec::HEADS * tc_dec::LAT * 4);
-  bf* u_merged = reinterpret_cast<bf*>(p);
   CUtensorMap mC, mQ;
   // Rows of the cache map: every row a tile reads lies inside some sequence
   // (the last tile of a sequence is shifted back to end at its end), so
@@ -166,12 +183,19 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   sp.n_seq = n; sp.G = G; sp.offs = offs; sp.plan = plan; sp.cache = static_cast<const bf*>(cache);
   sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   sp.part_ml = part_ml; sp.part_u = part_u;
-  tc_dec::decode_split_kernel<<<G, 192, tc_dec::SMEM_BYTES, st>>>(mC, mQ, sp);
-  tc_dec::merge_kernel<<<(n * tc_dec::HEADS + 7) / 8, 256, 0, st>>>(n, G, plan, sp.scale_log2, part_ml, part_u, u_merged);
-  tc_dec::project_kernel<<<dim3(tc_dec::HEADS, 128 / tc_dec::PRJ_Q, (n + tc_dec::PRJ_SEQ - 1) / tc_dec::PRJ_SEQ), 256,
-                           tc_dec::PRJ_SMEM, st>>>(
-      n, u_merged, static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate), static_cast<bf*>(O));
-  note_launches(4);
+  // The split and merge kernels are launched behind their predecessor
+  // (programmatic dependent launch): each waits for it with griddepcontrol.wait
+  // before touching its results, so only their set-up overlaps its tail.
+  GMLA_TRY(check_launch());
+  GMLA_TRY(cuda_status(launch_after_prev(tc_dec::decode_split_kernel, dim3(G), dim3(192), tc_dec::SMEM_BYTES, st,
+                                         mC, mQ, sp)));
+  GMLA_TRY(cuda_status(launch_after_prev(tc_dec::merge_project_kernel,
+                                         dim3(tc_dec::HEADS, (n + tc_dec::MP_SEQ - 1) / tc_dec::MP_SEQ),
+                                         dim3(tc_dec::MP_THREADS), tc_dec::MP_SMEM, st, n, G, (const int*)plan,
+                                         sp.scale_log2, (const float*)part_ml, (const float*)part_u,
+                                         static_cast<const bf*>(W_UKV), static_cast<const bf*>(gate),
+                                         static_cast<bf*>(O))));
+  note_launches(3);
   return check_launch();
 }
 

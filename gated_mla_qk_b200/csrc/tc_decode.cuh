@@ -65,7 +65,13 @@ enum Bar { QFULL = 0, QEMPTY, LFULL, LEMPTY = LFULL + NPS, RFULL = LEMPTY + NPS,
            PVDONE, UFREE, DRAIN, NBAR };
 
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kPrefetchAhead = 3;          // tiles brought into L2 ahead of their first ring load
+#ifndef GMLA_DEC_PF
+#define GMLA_DEC_PF 1
+#endif
+#ifndef GMLA_DEC_HINT
+#define GMLA_DEC_HINT 1
+#endif
+constexpr int kPrefetchAhead = GMLA_DEC_PF;   // tiles brought into L2 ahead of their first ring load
 
 struct SplitParams {
   int n_seq, G;
@@ -117,6 +123,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
 
+  // Launched behind the absorb kernel: q~ and the plan are its results.
+  griddep_wait();
+  griddep_launch_dependents();
   int nt, i0, k0;
   cta_range(p.plan, p.n_seq, p.G, cta, nt, i0, k0);
   if (nt == 0) return;                                   // whole CTA: empty range
@@ -162,18 +171,28 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
       };
       int u = 0, seg = 0, rope_issued = 0;
       bool ok = true;
-      auto load_pair = [&](int row, int pr) {
+#if GMLA_DEC_HINT
+      const uint64_t pol_keep = l2_policy_evict_last(), pol_drop = l2_policy_evict_first();
+#endif
+      auto load_pair = [&](int row, int pr, bool second) {
         const uint32_t slot = (uint32_t)(u % NPS);
         if (!mbar_wait(bar(LEMPTY + slot), ((uint32_t)(u / NPS) & 1u) ^ 1u, abort)) { ok = false; return; }
         const uint32_t dst = sbase + OFF_PAIR + slot * PAIR;
         mbar_arrive_expect_tx(bar(LFULL + slot), PAIR);
+#if GMLA_DEC_HINT
+        const uint64_t pol = second ? pol_drop : pol_keep;
+        tma_load_2d_hint(dst, &tmC, bar(LFULL + slot), 128 * pr, row, pol);
+        tma_load_2d_hint(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row, pol);
+#else
+        (void)second;
         tma_load_2d(dst, &tmC, bar(LFULL + slot), 128 * pr, row);
         tma_load_2d(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row);
+#endif
         ++u;
       };
       auto load_qk = [&](int t) {           // score-product items of tile t (cursor cq at t)
         const int row = cq.row();
-        for (int pr = 0; pr < 4 && ok; ++pr) load_pair(row, pr);
+        for (int pr = 0; pr < 4 && ok; ++pr) load_pair(row, pr, false);
         if (!ok) return;
         if (!mbar_wait(bar(REMPTY), ((uint32_t)t & 1u) ^ 1u, abort)) { ok = false; return; }
         mbar_arrive_expect_tx(bar(RFULL), CSUB);
@@ -197,7 +216,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
           load_qk(t + 1);
         }
         const int row = cp.row();
-        for (int pr = 0; pr < 4 && ok; ++pr) load_pair(row, pr);
+        for (int pr = 0; pr < 4 && ok; ++pr) load_pair(row, pr, true);
         cp.next();
         prefetch_upto(t + 2 + kPrefetchAhead);
       }
@@ -493,6 +512,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
   const int h = blockIdx.x, n0 = blockIdx.y * ABS_Q, i0 = blockIdx.z * ABS_SEQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   constexpr size_t ldw = (size_t)HEADS * 256;
+  griddep_launch_dependents();                 // the split kernel may be scheduled (it waits for this grid)
   if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) build_plan(n_seq, offs, G, plan);
   for (int e = threadIdx.x; e < ABS_Q * 16; e += blockDim.x) {
     const int n = e >> 4, c = e & 15;
@@ -539,110 +559,116 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
   }
 }
 
-// Merge the pieces of each (sequence, head): one warp per pair, 16 latents per
-// lane.  u = sum_s U_s 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c), in bf16.
-// The pieces of sequence i are those of the CTAs whose tile ranges meet the
-// sequence's tiles; CTA c's piece of sequence i is partial c + i.
-__global__ void __launch_bounds__(256) merge_kernel(int n_seq, int G, const int* __restrict__ plan, float scale_log2,
-                                                    const float* __restrict__ part_ml, const float* __restrict__ part_u,
-                                                    __nv_bfloat16* __restrict__ u_out) {
-  const int pair = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (pair >= n_seq * HEADS) return;
-  const int i = pair / HEADS, h = pair % HEADS;
-  const long long N = plan[n_seq];
-  const long long t_lo = plan[i], t_hi = plan[i + 1] - 1;
-  __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(u_out + ((size_t)i * HEADS + h) * LAT);
-  if (t_hi < t_lo) {                         // no tiles (outside the API's contract): zeros
-#pragma unroll
-    for (int q = 0; q < 8; ++q) dst[lane + 32 * q] = __floats2bfloat162_rn(0.f, 0.f);
-    return;
-  }
-  // CTA holding tile t: the largest c with floor(c N / G) <= t.
-  const int c_lo = (int)(((t_lo + 1) * G - 1) / N), c_hi = (int)(((t_hi + 1) * G - 1) / N);
-  auto empty = [&](int cc) { return (long long)cc * N / G == (long long)(cc + 1) * N / G; };
-  float M = -INFINITY;
-  for (int cc = c_lo; cc <= c_hi; ++cc)
-    if (!empty(cc)) M = fmaxf(M, part_ml[((size_t)(cc + i) * HEADS + h) * 2]);
-  float4 acc[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float Ls = 0.f;
-  for (int cc = c_lo; cc <= c_hi; ++cc) {
-    if (empty(cc)) continue;
-    const size_t k = (size_t)(cc + i) * HEADS + h;
-    const float w = ex2((part_ml[2 * k] - M) * scale_log2);
-    Ls += part_ml[2 * k + 1] * w;
-    const float4* src = reinterpret_cast<const float4*>(part_u + k * LAT);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = src[lane + 32 * q];
-      acc[q].x = fmaf(v.x, w, acc[q].x); acc[q].y = fmaf(v.y, w, acc[q].y);
-      acc[q].z = fmaf(v.z, w, acc[q].z); acc[q].w = fmaf(v.w, w, acc[q].w);
-    }
-  }
-  const float inv = 1.f / Ls;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int l4 = lane + 32 * q;
-    dst[2 * l4] = __floats2bfloat162_rn(acc[q].x * inv, acc[q].y * inv);
-    dst[2 * l4 + 1] = __floats2bfloat162_rn(acc[q].z * inv, acc[q].w * inv);
-  }
-}
+constexpr int MP_SEQ = 64;                     // sequences per merge + projection block
+constexpr int MP_THREADS = 1024;
+constexpr int LDU = LAT + 8;                   // padded bf16 row of a staged merged latent
+constexpr int LDWV = 128 + 8;                  // padded bf16 row of the staged W_UV,h
+constexpr size_t MP_SMEM = (size_t)LAT * LDWV * 2 + (size_t)MP_SEQ * LDU * 2;
 
-constexpr int PRJ_SEQ = 64;                    // sequences per projection block
-constexpr int PRJ_Q = 32;                      // output columns per projection block
-constexpr int LDU = LAT + 8;                   // padded bf16 row of the staged latent tile
-constexpr int LDWQ = PRJ_Q + 8;                // padded bf16 row of the staged W_UV,h columns
-constexpr size_t PRJ_SMEM = (size_t)LAT * LDWQ * 2 + (size_t)PRJ_SEQ * LDU * 2;
-
-// o[i][h] = u[i][h] W_UV,h (* sigmoid(g)).  Block = (head h, 32 output
-// columns, 64 sequences), 8 warps; warp w owns 8 output columns of 32
-// sequences.  The block's columns of W_UV,h (512 x 32, row-major) and its
-// merged latents are staged with cp.async; W_UV,h feeds the MMA through
-// transposing matrix loads.
-__global__ void __launch_bounds__(256) project_kernel(int n_seq, const __nv_bfloat16* __restrict__ u_in,
-                                                      const __nv_bfloat16* __restrict__ W_UKV,
-                                                      const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ O) {
-  extern __shared__ __align__(16) uint8_t csm[];
-  __nv_bfloat16* Wv = reinterpret_cast<__nv_bfloat16*>(csm);                    // [512][LDWQ]
-  __nv_bfloat16* U = Wv + LAT * LDWQ;                                            // [64][LDU]
-  const int h = blockIdx.x, q0 = blockIdx.y * PRJ_Q, i0 = blockIdx.z * PRJ_SEQ;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, t = lane & 3;
+// Merge + un-absorb, one block per (head h, 64 sequences), 32 warps.
+//   1. W_UV,h (512 x 128) is staged in shared memory with cp.async; it does
+//      not depend on the split kernel, so with a programmatic launch it is
+//      fetched while the split kernel finishes.
+//   2. Merge: the pieces of sequence i are those of the CTAs whose tile ranges
+//      meet the sequence's tiles (CTA c's piece of sequence i is partial c + i);
+//      u = sum_s U_s 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c), one warp per
+//      sequence, 16 latents per lane, rounded to bf16 into shared memory.
+//   3. o = u W_UV,h (* sigmoid(g)) with mma.sync: warp w owns 16 sequences
+//      (w mod 4) and 16 output columns (w / 4).
+__global__ void __launch_bounds__(MP_THREADS, 1)
+merge_project_kernel(int n_seq, int G, const int* __restrict__ plan, float scale_log2,
+                     const float* __restrict__ part_ml, const float* __restrict__ part_u,
+                     const __nv_bfloat16* __restrict__ W_UKV, const __nv_bfloat16* __restrict__ g,
+                     __nv_bfloat16* __restrict__ O) {
+  extern __shared__ __align__(16) uint8_t mps[];
+  __nv_bfloat16* Wv = reinterpret_cast<__nv_bfloat16*>(mps);                     // [512][LDWV]
+  __nv_bfloat16* Us = Wv + LAT * LDWV;                                             // [64][LDU]
+  const int h = blockIdx.x, i0 = blockIdx.y * MP_SEQ;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr size_t ldw = (size_t)HEADS * 256;
-  for (int e = threadIdx.x; e < LAT * (PRJ_Q / 8); e += blockDim.x) {
-    const int k = e / (PRJ_Q / 8), c = e % (PRJ_Q / 8);
-    cp_async16(Wv + k * LDWQ + c * 8, W_UKV + (size_t)k * ldw + (size_t)h * 256 + 128 + q0 + c * 8);
+  for (int e = threadIdx.x; e < LAT * 16; e += MP_THREADS) {
+    const int k = e >> 4, c = e & 15;
+    cp_async16(Wv + k * LDWV + c * 8, W_UKV + (size_t)k * ldw + (size_t)h * 256 + 128 + c * 8);
   }
-  for (int e = threadIdx.x; e < PRJ_SEQ * (LAT / 8); e += blockDim.x) {
-    const int r = e / (LAT / 8), c = e % (LAT / 8), i = i0 + r;
-    if (i < n_seq) cp_async16(U + r * LDU + c * 8, u_in + ((size_t)i * HEADS + h) * LAT + c * 8);
-    else *reinterpret_cast<uint4*>(U + r * LDU + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+  griddep_wait();                                // the split kernel's partials
+  const long long N = plan[n_seq];
+  auto empty = [&](int cc) { return (long long)cc * N / G == (long long)(cc + 1) * N / G; };
+  for (int r = warp; r < MP_SEQ; r += MP_THREADS / 32) {
+    const int i = i0 + r;
+    uint2* dst = reinterpret_cast<uint2*>(Us + r * LDU);
+    const long long t_lo = i < n_seq ? plan[i] : 0, t_hi = i < n_seq ? plan[i + 1] - 1 : -1;
+    if (t_hi < t_lo) {                         // padding row, or a sequence with no tiles: zeros
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[lane + 32 * q] = make_uint2(0u, 0u);
+      continue;
+    }
+    // CTA holding tile t: the largest c with floor(c N / G) <= t.
+    const int c_lo = (int)(((t_lo + 1) * G - 1) / N), c_hi = (int)(((t_hi + 1) * G - 1) / N);
+    float M = -INFINITY;
+    for (int cc = c_lo + lane; cc <= c_hi; cc += 32)
+      if (!empty(cc)) M = fmaxf(M, part_ml[((size_t)(cc + i) * HEADS + h) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float4 acc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Ls = 0.f;
+    for (int base = c_lo; base <= c_hi; base += 32) {
+      const int cnt = min(32, c_hi - base + 1);
+      float wl = 0.f, ll = 0.f;                // lane j: weight and weighted sum of piece base + j
+      if (lane < cnt && !empty(base + lane)) {
+        const size_t k = (size_t)(base + lane + i) * HEADS + h;
+        wl = ex2((part_ml[2 * k] - M) * scale_log2);
+        ll = part_ml[2 * k + 1] * wl;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
+      Ls += ll;
+#pragma unroll 4
+      for (int j = 0; j < cnt; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wl, j);
+        // An empty piece (weight 0) was never written: its partial is not read.
+        const float4* src = reinterpret_cast<const float4*>(part_u + ((size_t)(base + j + i) * HEADS + h) * LAT);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = w != 0.f ? src[lane + 32 * q] : make_float4(0.f, 0.f, 0.f, 0.f);
+          acc[q].x = fmaf(v.x, w, acc[q].x); acc[q].y = fmaf(v.y, w, acc[q].y);
+          acc[q].z = fmaf(v.z, w, acc[q].z); acc[q].w = fmaf(v.w, w, acc[q].w);
+        }
+      }
+    }
+    const float inv = 1.f / Ls;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[lane + 32 * q] = make_uint2(pack_bf16x2(acc[q].x * inv, acc[q].y * inv),
+                                      pack_bf16x2(acc[q].z * inv, acc[q].w * inv));
   }
   cp_async_wait_all();
   __syncthreads();
-  const int nt = warp & 3, mt0 = (warp >> 2) * 2;
+  const int gq = lane >> 2, t = lane & 3;
+  const int mt = warp & 3, c0 = (warp >> 2) * 16;
   float acc[2][4] = {};
 #pragma unroll 4
   for (int kk = 0; kk < LAT / 16; ++kk) {
     const int k0 = kk * 16;
-    uint32_t b0, b1;
-    ldsm_x2_trans(b0, b1, Wv + (k0 + (lane & 15)) * LDWQ + nt * 8);
+    const __nv_bfloat16* ar = Us + (mt * 16 + gq) * LDU + k0 + 2 * t;
+    const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDU), lds32(ar + 8), lds32(ar + 8 * LDU + 8)};
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const __nv_bfloat16* ar = U + ((mt0 + m) * 16 + gq) * LDU + k0 + 2 * t;
-      const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDU), lds32(ar + 8), lds32(ar + 8 * LDU + 8)};
-      mma16816(acc[m], a, b0, b1);
+    for (int nt = 0; nt < 2; ++nt) {
+      uint32_t b0, b1;
+      ldsm_x2_trans(b0, b1, Wv + (k0 + (lane & 15)) * LDWV + c0 + nt * 8);
+      mma16816(acc[nt], a, b0, b1);
     }
   }
 #pragma unroll
-  for (int m = 0; m < 2; ++m)
+  for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
-      const int i = i0 + (mt0 + m) * 16 + gq + 8 * hr;
+      const int i = i0 + mt * 16 + gq + 8 * hr;
       if (i >= n_seq) continue;
-      const int col = q0 + nt * 8 + 2 * t;
+      const int col = c0 + nt * 8 + 2 * t;
       const size_t idx = ((size_t)i * HEADS + h) * 128 + col;
-      float o0 = acc[m][2 * hr], o1 = acc[m][2 * hr + 1];
+      float o0 = acc[nt][2 * hr], o1 = acc[nt][2 * hr + 1];
       if (g) {
         const float2 gv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(g + idx));
         o0 *= 1.f / (1.f + __expf(-gv.x));
@@ -657,7 +683,7 @@ inline size_t workspace_bytes(int n) {
   auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
   const size_t np = (size_t)G_CAP + n;
   return al((size_t)n * HEADS * WID * 2) + al(((size_t)n + 1 + G_CAP) * 4) + al(np * HEADS * 2 * 4) +
-         al(np * HEADS * LAT * 4) + al((size_t)n * HEADS * LAT * 2);
+         al(np * HEADS * LAT * 4);
 }
 
 }  // namespace tc_dec
