@@ -79,6 +79,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// The same wait with one inline try_wait and the bounded loop out of line, for
+// a thread that issues MMAs: its common case (the phase has already completed)
+// stays a few instructions long.
+__device__ __noinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait(bar, parity, abort);
+}
+__device__ __forceinline__ bool mbar_wait_lean(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_loop(bar, parity, abort);
+}
+
 // Drain wait, used before a CTA exits: waits for this CTA's own copies or
 // MMAs still in flight, ignoring abort requests, bounded by kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
@@ -338,6 +349,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= (uint64_t)2 << 61;
   return d;
 }
+
+// A descriptor moved by `bytes` (a multiple of 16).  The start-address field
+// holds address >> 4 in its low 14 bits; shared-memory addresses stay below
+// 256 KB, so the add never carries out of the field.  An issuing thread can
+// build a few base descriptors once and step them with this add.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 // Bits: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,

@@ -233,46 +233,57 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
       bool ok = true;
       int u = 0;
       auto wait_ok = [&](int b, uint32_t ph) {
-        ok = ok && mbar_wait(bar(b), ph, abort);
+        ok = ok && mbar_wait_lean(bar(b), ph, abort);
         if (ok) tc_fence_after();
         return ok;
       };
-      auto next_pair = [&]() -> uint32_t {    // wait for ring item u; returns its slot address
-        const uint32_t slot = (uint32_t)(u % NPS);
-        if (!wait_ok(LFULL + slot, (uint32_t)(u / NPS) & 1u)) return 0;
-        return sbase + OFF_PAIR + slot * PAIR;
+      // Base descriptors, built once: every MMA below steps one of them by a
+      // compile-time byte offset (or picks a ring slot's).
+      const uint64_t dQ = sdesc_sw128(sbase + OFF_Q, 16, 1024);
+      const uint64_t dRope = sdesc_sw128(sbase + OFF_ROPE, 16, 1024);
+      const uint64_t dP = sdesc_sw128(sbase + OFF_P, 16, 1024);
+      const uint64_t dRingK = sdesc_sw128(sbase + OFF_PAIR, 16, 1024);     // slot 0, K-major (score B)
+      const uint64_t dRingM = sdesc_sw128(sbase + OFF_PAIR, CSUB, 1024);   // slot 0, MN-major (value A)
+      int slot_u = 0;                          // u % NPS and (u / NPS) & 1, kept incrementally
+      uint32_t ph_u = 0;
+      auto next_pair = [&]() -> bool {         // wait for ring item u
+        return wait_ok(LFULL + slot_u, ph_u);
       };
-      auto release_pair = [&]() { mma_commit(bar(LEMPTY + u % NPS)); ++u; };
+      auto release_pair = [&]() {
+        mma_commit(bar(LEMPTY + slot_u));
+        ++u;
+        if (++slot_u == NPS) { slot_u = 0; ph_u ^= 1u; }
+      };
       auto qk = [&](int t) {
         const uint32_t d = tmem + TM_S;
+#pragma unroll 1
         for (int q = 0; q < 4; ++q) {
-          const uint32_t sb = next_pair();
-          if (!ok) return;
+          if (!next_pair()) return;
+          const uint64_t sb = sdesc_add(dRingK, (uint32_t)slot_u * PAIR);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_ss(d, sdesc_sw128(sbase + OFF_Q + (uint32_t)(2 * q + hf) * QCH + kk * 32u, 16, 1024),
-                     sdesc_sw128(sb + hf * CSUB + kk * 32u, 16, 1024), idQK, (q | hf | kk) != 0);
+              mma_ss(d, sdesc_add(dQ, (uint32_t)(2 * q + hf) * QCH + kk * 32u), sdesc_add(sb, hf * CSUB + kk * 32u), idQK,
+                     (q | hf | kk) != 0);
           release_pair();
         }
         if (!wait_ok(RFULL, (uint32_t)t & 1u)) return;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(d, sdesc_sw128(sbase + OFF_Q + 8u * QCH + kk * 32u, 16, 1024),
-                 sdesc_sw128(sbase + OFF_ROPE + kk * 32u, 16, 1024), idQK, true);
+          mma_ss(d, sdesc_add(dQ, 8u * QCH + kk * 32u), sdesc_add(dRope, kk * 32u), idQK, true);
         mma_commit(bar(REMPTY));
         mma_commit(bar(SFULL));
       };
       auto pv = [&](bool fresh) {
+#pragma unroll 1
         for (int b = 0; b < 4; ++b) {
-          const uint32_t sb = next_pair();
-          if (!ok) return;
+          if (!next_pair()) return;
+          const uint64_t sb = sdesc_add(dRingM, (uint32_t)slot_u * PAIR);
 #pragma unroll
           for (int kk = 0; kk < BT / 16; ++kk)
-            mma_ss(tmem + TM_U + (uint32_t)b * HEADS, sdesc_sw128(sb + kk * 2048u, CSUB, 1024),
-                   sdesc_sw128(sbase + OFF_P + (uint32_t)(kk >> 2) * QCH + (uint32_t)(kk & 3) * 32u, 16, 1024), idPV,
-                   !(fresh && kk == 0));
+            mma_ss(tmem + TM_U + (uint32_t)b * HEADS, sdesc_add(sb, kk * 2048u),
+                   sdesc_add(dP, (uint32_t)(kk >> 2) * QCH + (uint32_t)(kk & 3) * 32u), idPV, !(fresh && kk == 0));
           release_pair();
         }
         mma_commit(bar(PVDONE));
