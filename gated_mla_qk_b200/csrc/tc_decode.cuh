@@ -571,21 +571,41 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
 }
 
 constexpr int MP_SEQ = 64;                     // sequences per merge + projection block
-constexpr int MP_THREADS = 1024;
+constexpr int MP_THREADS = 512;
+constexpr int MP_MAXP = 32;                    // pieces per sequence merged in one batch
 constexpr int LDU = LAT + 8;                   // padded bf16 row of a staged merged latent
 constexpr int LDWV = 128 + 8;                  // padded bf16 row of the staged W_UV,h
 constexpr size_t MP_SMEM = (size_t)LAT * LDWV * 2 + (size_t)MP_SEQ * LDU * 2;
 
-// Merge + un-absorb, one block per (head h, 64 sequences), 32 warps.
+// Pieces of one sequence for the merge: CTA c's piece of sequence i is
+// partial c + i, for the CTAs c in [c_lo, c_hi] whose tile ranges meet the
+// sequence's tiles (empty ranges write nothing and are skipped).
+struct MergeSeq {
+  int i, c_lo, n;                              // n = 0: no tiles (zeros)
+  __device__ void init(int seq, int n_seq, int G, const int* plan, long long N) {
+    i = seq;
+    n = 0;
+    c_lo = 0;
+    if (seq >= n_seq) return;
+    const long long t_lo = plan[seq], t_hi = plan[seq + 1] - 1;
+    if (t_hi < t_lo) return;
+    // CTA holding tile t: the largest c with floor(c N / G) <= t.
+    c_lo = (int)(((t_lo + 1) * G - 1) / N);
+    n = (int)(((t_hi + 1) * G - 1) / N) - c_lo + 1;
+  }
+};
+
+// Merge + un-absorb, one block per (head h, 64 sequences), 16 warps.
 //   1. W_UV,h (512 x 128) is staged in shared memory with cp.async; it does
 //      not depend on the split kernel, so with a programmatic launch it is
 //      fetched while the split kernel finishes.
-//   2. Merge: the pieces of sequence i are those of the CTAs whose tile ranges
-//      meet the sequence's tiles (CTA c's piece of sequence i is partial c + i);
-//      u = sum_s U_s 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c), one warp per
-//      sequence, 16 latents per lane, rounded to bf16 into shared memory.
+//   2. Merge: u = sum_s U_s 2^((m_s - M) c) / sum_s l_s 2^((m_s - M) c) over
+//      the pieces s of a sequence, rounded to bf16 into shared memory.  A warp
+//      merges two sequences at a time: lane j reads piece j's (m, l) of both,
+//      then the pieces' U rows (16 latents per lane) of both sequences are
+//      loaded together, so each pair costs two dependent global round trips.
 //   3. o = u W_UV,h (* sigmoid(g)) with mma.sync: warp w owns 16 sequences
-//      (w mod 4) and 16 output columns (w / 4).
+//      (w mod 4) and 32 output columns (w / 4).
 __global__ void __launch_bounds__(MP_THREADS, 1)
 merge_project_kernel(int n_seq, int G, const int* __restrict__ plan, float scale_log2,
                      const float* __restrict__ part_ml, const float* __restrict__ part_u,
@@ -604,75 +624,102 @@ merge_project_kernel(int n_seq, int G, const int* __restrict__ plan, float scale
   griddep_wait();                                // the split kernel's partials
   const long long N = plan[n_seq];
   auto empty = [&](int cc) { return (long long)cc * N / G == (long long)(cc + 1) * N / G; };
-  for (int r = warp; r < MP_SEQ; r += MP_THREADS / 32) {
-    const int i = i0 + r;
-    uint2* dst = reinterpret_cast<uint2*>(Us + r * LDU);
-    const long long t_lo = i < n_seq ? plan[i] : 0, t_hi = i < n_seq ? plan[i + 1] - 1 : -1;
-    if (t_hi < t_lo) {                         // padding row, or a sequence with no tiles: zeros
+  for (int r0 = warp; r0 < MP_SEQ; r0 += 2 * (MP_THREADS / 32)) {
+    MergeSeq sq[2];
+    sq[0].init(i0 + r0, n_seq, G, plan, N);
+    sq[1].init(i0 + r0 + MP_THREADS / 32, n_seq, G, plan, N);
+    float4 acc[2][4];
+    float Ls[2] = {0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) dst[lane + 32 * q] = make_uint2(0u, 0u);
-      continue;
-    }
-    // CTA holding tile t: the largest c with floor(c N / G) <= t.
-    const int c_lo = (int)(((t_lo + 1) * G - 1) / N), c_hi = (int)(((t_hi + 1) * G - 1) / N);
-    float M = -INFINITY;
-    for (int cc = c_lo + lane; cc <= c_hi; cc += 32)
-      if (!empty(cc)) M = fmaxf(M, part_ml[((size_t)(cc + i) * HEADS + h) * 2]);
+    for (int a = 0; a < 2; ++a)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float4 acc[4];
+      for (int q = 0; q < 4; ++q) acc[a][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int nmax = max(sq[0].n, sq[1].n);
+    for (int base = 0; base < nmax; base += MP_MAXP) {
+      // Lane j: (m, l) of piece base + j of both sequences, one round trip.
+      float ml[2], ll[2], M[2], w[2];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Ls = 0.f;
-    for (int base = c_lo; base <= c_hi; base += 32) {
-      const int cnt = min(32, c_hi - base + 1);
-      float wl = 0.f, ll = 0.f;                // lane j: weight and weighted sum of piece base + j
-      if (lane < cnt && !empty(base + lane)) {
-        const size_t k = (size_t)(base + lane + i) * HEADS + h;
-        wl = ex2((part_ml[2 * k] - M) * scale_log2);
-        ll = part_ml[2 * k + 1] * wl;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
-      Ls += ll;
-#pragma unroll 4
-      for (int j = 0; j < cnt; ++j) {
-        const float w = __shfl_sync(0xffffffffu, wl, j);
-        // An empty piece (weight 0) was never written: its partial is not read.
-        const float4* src = reinterpret_cast<const float4*>(part_u + ((size_t)(base + j + i) * HEADS + h) * LAT);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 v = w != 0.f ? src[lane + 32 * q] : make_float4(0.f, 0.f, 0.f, 0.f);
-          acc[q].x = fmaf(v.x, w, acc[q].x); acc[q].y = fmaf(v.y, w, acc[q].y);
-          acc[q].z = fmaf(v.z, w, acc[q].z); acc[q].w = fmaf(v.w, w, acc[q].w);
+      for (int a = 0; a < 2; ++a) {
+        ml[a] = -INFINITY; ll[a] = 0.f;
+        const int cc = sq[a].c_lo + base + lane;
+        if (base + lane < sq[a].n && !empty(cc)) {
+          const size_t k = (size_t)(cc + sq[a].i) * HEADS + h;
+          ml[a] = part_ml[2 * k];
+          ll[a] = part_ml[2 * k + 1];
         }
       }
-    }
-    const float inv = 1.f / Ls;
+      // A sequence with more than MP_MAXP pieces needs the max over all of
+      // them before any weight: take it from a first pass in that case.
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      dst[lane + 32 * q] = make_uint2(pack_bf16x2(acc[q].x * inv, acc[q].y * inv),
-                                      pack_bf16x2(acc[q].z * inv, acc[q].w * inv));
+      for (int a = 0; a < 2; ++a) {
+        M[a] = ml[a];
+        if (sq[a].n > MP_MAXP)
+          for (int cc = sq[a].c_lo + lane; cc < sq[a].c_lo + sq[a].n; cc += 32)
+            if (!empty(cc)) M[a] = fmaxf(M[a], part_ml[((size_t)(cc + sq[a].i) * HEADS + h) * 2]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M[a] = fmaxf(M[a], __shfl_xor_sync(0xffffffffu, M[a], o));
+        // Empty or missing pieces have m = -inf, hence weight 0.
+        w[a] = ml[a] == -INFINITY ? 0.f : ex2((ml[a] - M[a]) * scale_log2);
+        float lw = ll[a] * w[a];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+        Ls[a] += lw;
+      }
+      const int cnt = min(MP_MAXP, nmax - base);
+#pragma unroll 2
+      for (int j = 0; j < cnt; ++j) {
+        float4 v[2][4];
+        float wj[2];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          wj[a] = __shfl_sync(0xffffffffu, w[a], j);
+          // A piece with weight 0 (empty, or past this sequence's pieces) is not read.
+          const float4* src = reinterpret_cast<const float4*>(
+              part_u + ((size_t)(sq[a].c_lo + base + j + sq[a].i) * HEADS + h) * LAT);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) v[a][q] = wj[a] != 0.f ? src[lane + 32 * q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[a][q].x = fmaf(v[a][q].x, wj[a], acc[a][q].x); acc[a][q].y = fmaf(v[a][q].y, wj[a], acc[a][q].y);
+            acc[a][q].z = fmaf(v[a][q].z, wj[a], acc[a][q].z); acc[a][q].w = fmaf(v[a][q].w, wj[a], acc[a][q].w);
+          }
+      }
+      // With more than MP_MAXP pieces, later batches must use the same M:
+      // the first pass above already took the max over all pieces.
+    }
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const int r = r0 + a * (MP_THREADS / 32);
+      uint2* dst = reinterpret_cast<uint2*>(Us + r * LDU);
+      const float inv = sq[a].n > 0 ? 1.f / Ls[a] : 0.f;   // no tiles: zeros
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[lane + 32 * q] = make_uint2(pack_bf16x2(acc[a][q].x * inv, acc[a][q].y * inv),
+                                        pack_bf16x2(acc[a][q].z * inv, acc[a][q].w * inv));
+    }
   }
   cp_async_wait_all();
   __syncthreads();
   const int gq = lane >> 2, t = lane & 3;
-  const int mt = warp & 3, c0 = (warp >> 2) * 16;
-  float acc[2][4] = {};
+  const int mt = warp & 3, c0 = (warp >> 2) * 32;
+  float acc[4][4] = {};
 #pragma unroll 4
   for (int kk = 0; kk < LAT / 16; ++kk) {
     const int k0 = kk * 16;
     const __nv_bfloat16* ar = Us + (mt * 16 + gq) * LDU + k0 + 2 * t;
     const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * LDU), lds32(ar + 8), lds32(ar + 8 * LDU + 8)};
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < 4; ++nt) {
       uint32_t b0, b1;
       ldsm_x2_trans(b0, b1, Wv + (k0 + (lane & 15)) * LDWV + c0 + nt * 8);
       mma16816(acc[nt], a, b0, b1);
     }
   }
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const int i = i0 + mt * 16 + gq + 8 * hr;
