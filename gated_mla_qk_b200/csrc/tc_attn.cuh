@@ -20,7 +20,8 @@
 // O accumulator at [256,384).
 // Shared memory (1024-aligned, 128B-swizzled 16 KB sub-tiles of 128 x 64 bf16):
 //   Q: 3 sub-tiles (q^C 0-63, q^C 64-127, q^S) | ring: 3 slots x 3 sub-tiles
-//   (K slot = K^C 0-63, K^C 64-127, k^S; V slot = V 0-63, V 64-127) | P: 2.
+//   (K slot = K^C 0-63, K^C 64-127, k^S; V slot = V 0-63, V 64-127).  P never
+//   goes through shared memory: it is written into TMEM over its S buffer.
 // Softmax uses base-2 exponentials of the scaled logits with a lazily
 // updated reference max: O and l are rescaled only when a row's max grows by
 // more than a factor 2^8, which keeps every exponential <= 256 and is exact
@@ -39,8 +40,7 @@ constexpr int NSTAGE = 3;
 constexpr uint32_t SUB = 128 * 128;                       // bytes of one 128 x 64 bf16 sub-tile
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_RING = OFF_Q + 3 * SUB;
-constexpr uint32_t OFF_P = OFF_RING + NSTAGE * 3 * SUB;
-constexpr uint32_t OFF_BAR = OFF_P + 2 * SUB;
+constexpr uint32_t OFF_BAR = OFF_RING + NSTAGE * 3 * SUB;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;     // + barriers + alignment slack
 
 enum Bar { QFULL = 0, KVFULL = 1, KVEMPTY = KVFULL + NSTAGE, SFULL = KVEMPTY + NSTAGE, PFULL = SFULL + 2,
