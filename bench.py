@@ -93,7 +93,7 @@ def train_leg(args, gm, synth, geom, rank, st, dist):
         "attn_fwd_train_B1_T4096": {"ms": f_ms, "value": f_flop / (f_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                                     "what": "mla_attn_fwd_train (fp32 o, lse)"},
         "attn_bwd_B1_T4096": {"ms": b_ms, "value": b_flop / (b_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-                              "what": "mla_attn_bwd, warp-level bf16 tensor-core passes (mma.sync), fp32 accumulation",
+                              "what": "mla_attn_bwd: tcgen05 dK/dV and dQ kernels (bf16 operands, fp32 TMEM accumulation)",
                               "roofline": {"bound": "tensor", "peak": pk_bf16, "unit": "TFLOP/s",
                                            "frac": b_flop / (b_ms / 1e3) / 1e12 / pk_bf16}},
     }

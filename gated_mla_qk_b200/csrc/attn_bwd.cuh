@@ -1,6 +1,7 @@
 // Backward of the causal gated MLA attention, CUDA-core form (fp32 arithmetic,
 // fp32 gradients; Q/K^C/k^S/V/g in the layer's dtype, o and dL/do in fp32 as
-// the training forward leaves them).
+// the training forward leaves them), for head widths other than Kimi K3's and
+// for fp32 layers.  The row pass below also serves the tcgen05 kernels.
 //
 // Forward ("Kimi K3 · Gated MLA · OpenModelAtlas", "All 20 steps"):
 //   S = Q_h K_h^T / sqrt(d_qk), K_h = [K^C_h | k^S];  A = causal softmax(S);
@@ -30,7 +31,7 @@ constexpr int BQ = 32, BK = 32, NT = 256;
 constexpr int kMaxD = 256;                       // d_qk and d_v limits
 
 // One warp per (b, t, h): D, dO~ and dg.
-// TO = float for the CUDA-core passes, bf16 for the tensor-core passes.
+// TO = float for the CUDA-core passes, bf16 for the tcgen05 kernels (tc_bwd.cuh).
 template <typename T, typename TO>
 __global__ void __launch_bounds__(256) row_kernel(int rows, int H, int d_v, const float* __restrict__ O,
                                                   const float* __restrict__ dO, const T* __restrict__ g,
@@ -218,249 +219,10 @@ __global__ void __launch_bounds__(NT) dq_kernel(Dims p, const T* __restrict__ Q,
   }
 }
 
-// ---------------------------------------------------------------------------
-// Tensor-core passes (bf16, d_c = 128, d_s = 64, d_v = 128): warp-level
-// mma.sync m16n8k16 with fp32 accumulators.  A block of four warps owns 64
-// rows (dQ pass: query rows; dK/dV pass: key rows), each warp 16 of them;
-// the other side streams through shared memory in 64-row tiles.  S, A, dA
-// and dS of a 16 x 64 piece stay in registers: the accumulator layout of two
-// adjacent n8 tiles is the A-operand layout of the next product, so A and dS
-// feed the dV, dK and dQ products without a trip through memory.  dO~ and A,
-// dS enter the products in bf16 (fp32 accumulation), like the forward's P.
-// ---------------------------------------------------------------------------
-namespace tc {
-
-using namespace sm100;
-
-constexpr int R = 64, DQK = 192, DV = 128, LQ = DQK + 8, LV = DV + 8;
-constexpr size_t SMEM = (size_t)(2 * R * LQ + 2 * R * LV) * 2 + 2 * R * 4;
-constexpr float kLog2e = 1.4426950408889634f;
-
-// Rows [r0, r0 + 64) (zero past T) of a head slice into dst[64][ld]:
-// `width` bf16 per row from src + ((b T + t) row_stride), as 16-byte cp.async.
-__device__ __forceinline__ void stage(__nv_bfloat16* dst, int ld, const __nv_bfloat16* src, size_t row_stride, int b,
-                                      int r0, int T_, int width) {
-  const int chunks = width / 8;
-  for (int e = threadIdx.x; e < R * chunks; e += 128) {
-    const int r = e / chunks, c = e - r * chunks, t = r0 + r;
-    if (t < T_) cp_async16(dst + r * ld + c * 8, src + ((size_t)b * T_ + t) * row_stride + c * 8);
-    else *reinterpret_cast<uint4*>(dst + r * ld + c * 8) = make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-// acc[8][4] (16 rows x 64 columns) += rows [m0, m0+16) of A (smem, [row][k],
-// ld) times the 64 rows of Bn (smem, [n][k], ld) over k in [0, K).
-template <int K>
-__device__ __forceinline__ void mm_nk(float (&acc)[8][4], const __nv_bfloat16* A, int lda, int m0,
-                                      const __nv_bfloat16* Bn, int ldb) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, tg = lane & 3;
-#pragma unroll
-  for (int ks = 0; ks < K / 16; ++ks) {
-    const __nv_bfloat16* ar = A + (m0 + g) * lda + ks * 16 + 2 * tg;
-    const uint32_t a[4] = {lds32(ar), lds32(ar + 8 * lda), lds32(ar + 8), lds32(ar + 8 * lda + 8)};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const __nv_bfloat16* br = Bn + (nt * 8 + g) * ldb + ks * 16 + 2 * tg;
-      mma16816(acc[nt], a, lds32(br), lds32(br + 8));
-    }
-  }
-}
-
-// acc[N/8][4] += P (16 x 64, as four A fragments) times rows [0, 64) of Bk
-// (smem, [k][n], ld), n in [0, N).
-template <int N>
-__device__ __forceinline__ void mm_kn(float (&acc)[N / 8][4], const uint32_t (&pa)[4][4], const __nv_bfloat16* Bk,
-                                      int ldb) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-    for (int nt = 0; nt < N / 8; ++nt) {
-      uint32_t b0, b1;
-      ldsm_x2_trans(b0, b1, Bk + (kk * 16 + (lane & 15)) * ldb + nt * 8);
-      mma16816(acc[nt], pa[kk], b0, b1);
-    }
-}
-
-// Accumulator pairs (n tiles 2kk, 2kk+1) -> bf16 A fragments.
-__device__ __forceinline__ void to_afrag(uint32_t (&pa)[4][4], const float (&x)[8][4]) {
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    pa[kk][0] = pack_bf16x2(x[2 * kk][0], x[2 * kk][1]);
-    pa[kk][1] = pack_bf16x2(x[2 * kk][2], x[2 * kk][3]);
-    pa[kk][2] = pack_bf16x2(x[2 * kk + 1][0], x[2 * kk + 1][1]);
-    pa[kk][3] = pack_bf16x2(x[2 * kk + 1][2], x[2 * kk + 1][3]);
-  }
-}
-
-__device__ __forceinline__ void stage_k(__nv_bfloat16* Ks, const __nv_bfloat16* KC, const __nv_bfloat16* kS, int b,
-                                        int h, int H, int k0, int T_) {
-  stage(Ks, LQ, KC + (size_t)h * 128, (size_t)H * 128, b, k0, T_, 128);
-  stage(Ks + 128, LQ, kS, 64, b, k0, T_, 64);
-}
-
-// Block = (query tile, head, batch), longest causal rows first: dQ_h.
-__global__ void __launch_bounds__(128) dq_kernel(Dims p, const __nv_bfloat16* __restrict__ Q,
-                                                 const __nv_bfloat16* __restrict__ KC,
-                                                 const __nv_bfloat16* __restrict__ kS,
-                                                 const __nv_bfloat16* __restrict__ V, const float* __restrict__ lse,
-                                                 const __nv_bfloat16* __restrict__ dOt, const float* __restrict__ D,
-                                                 float* __restrict__ dQ) {
-  extern __shared__ __align__(16) uint8_t smb[];
-  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smb);
-  __nv_bfloat16* Ks = Qs + R * LQ;
-  __nv_bfloat16* dOs = Ks + R * LQ;
-  __nv_bfloat16* Vs = dOs + R * LV;
-  const int H = p.H, T_ = p.T;
-  const int nqt = (T_ + R - 1) / R;
-  const int qt = nqt - 1 - (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z, q0 = qt * R;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tg = lane & 3;
-  stage(Qs, LQ, Q + (size_t)h * DQK, (size_t)H * DQK, b, q0, T_, DQK);
-  stage(dOs, LV, dOt + (size_t)h * DV, (size_t)H * DV, b, q0, T_, DV);
-  const int ra = q0 + warp * 16 + g, rb = ra + 8;
-  const float c = p.scale * kLog2e;
-  const float la = ra < T_ ? lse[((size_t)b * T_ + ra) * H + h] * kLog2e : 0.f;
-  const float lb = rb < T_ ? lse[((size_t)b * T_ + rb) * H + h] * kLog2e : 0.f;
-  const float Da = ra < T_ ? D[((size_t)b * T_ + ra) * H + h] : 0.f;
-  const float Db = rb < T_ ? D[((size_t)b * T_ + rb) * H + h] : 0.f;
-  float acc[DQK / 8][4];
-#pragma unroll
-  for (int i = 0; i < DQK / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  for (int kt = 0; kt <= qt; ++kt) {
-    const int k0 = kt * R;
-    __syncthreads();
-    stage_k(Ks, KC, kS, b, h, H, k0, T_);
-    stage(Vs, LV, V + (size_t)h * DV, (size_t)H * DV, b, k0, T_, DV);
-    cp_async_wait_all();
-    __syncthreads();
-    float S[8][4] = {}, dP[8][4] = {};
-    mm_nk<DQK>(S, Qs, LQ, warp * 16, Ks, LQ);
-    mm_nk<DV>(dP, dOs, LV, warp * 16, Vs, LV);
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = e < 2 ? ra : rb, key = k0 + nt * 8 + 2 * tg + (e & 1);
-        const float a = (key <= row && row < T_) ? exp2f(fmaf(S[nt][e], c, -(e < 2 ? la : lb))) : 0.f;
-        S[nt][e] = a * (dP[nt][e] - (e < 2 ? Da : Db));          // dS
-      }
-    uint32_t pa[4][4];
-    to_afrag(pa, S);
-    mm_kn<DQK>(acc, pa, Ks, LQ);
-  }
-#pragma unroll
-  for (int nt = 0; nt < DQK / 8; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int row = e < 2 ? ra : rb, col = nt * 8 + 2 * tg + (e & 1);
-      if (row < T_) dQ[(((size_t)b * T_ + row) * H + h) * DQK + col] = acc[nt][e] * p.scale;
-    }
-}
-
-// Block = (key tile, head, batch): dK^C_h, dV_h and this head's share of dk^S.
-__global__ void __launch_bounds__(128) dkdv_kernel(Dims p, const __nv_bfloat16* __restrict__ Q,
-                                                   const __nv_bfloat16* __restrict__ KC,
-                                                   const __nv_bfloat16* __restrict__ kS,
-                                                   const __nv_bfloat16* __restrict__ V, const float* __restrict__ lse,
-                                                   const __nv_bfloat16* __restrict__ dOt, const float* __restrict__ D,
-                                                   float* __restrict__ dKC, float* __restrict__ dkS,
-                                                   float* __restrict__ dV) {
-  extern __shared__ __align__(16) uint8_t smb[];
-  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smb);
-  __nv_bfloat16* Qs = Ks + R * LQ;
-  __nv_bfloat16* Vs = Qs + R * LQ;
-  __nv_bfloat16* dOs = Vs + R * LV;
-  float* slse = reinterpret_cast<float*>(dOs + R * LV);
-  float* sD = slse + R;
-  const int H = p.H, T_ = p.T;
-  const int nqt = (T_ + R - 1) / R;
-  const int kt = blockIdx.x, h = blockIdx.y, b = blockIdx.z, k0 = kt * R;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tg = lane & 3;
-  stage_k(Ks, KC, kS, b, h, H, k0, T_);
-  stage(Vs, LV, V + (size_t)h * DV, (size_t)H * DV, b, k0, T_, DV);
-  const int ka = k0 + warp * 16 + g, kb = ka + 8;
-  const float c = p.scale * kLog2e;
-  float aV[DV / 8][4], aK[DQK / 8][4];
-#pragma unroll
-  for (int i = 0; i < DV / 8; ++i) aV[i][0] = aV[i][1] = aV[i][2] = aV[i][3] = 0.f;
-#pragma unroll
-  for (int i = 0; i < DQK / 8; ++i) aK[i][0] = aK[i][1] = aK[i][2] = aK[i][3] = 0.f;
-  for (int qt = kt; qt < nqt; ++qt) {
-    const int q0 = qt * R;
-    __syncthreads();
-    stage(Qs, LQ, Q + (size_t)h * DQK, (size_t)H * DQK, b, q0, T_, DQK);
-    stage(dOs, LV, dOt + (size_t)h * DV, (size_t)H * DV, b, q0, T_, DV);
-    if (threadIdx.x < R) {
-      const int t = q0 + threadIdx.x;
-      slse[threadIdx.x] = t < T_ ? lse[((size_t)b * T_ + t) * H + h] * kLog2e : 0.f;
-      sD[threadIdx.x] = t < T_ ? D[((size_t)b * T_ + t) * H + h] : 0.f;
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    float St[8][4] = {}, dPt[8][4] = {};
-    mm_nk<DQK>(St, Ks, LQ, warp * 16, Qs, LQ);               // S^T: keys x queries
-    mm_nk<DV>(dPt, Vs, LV, warp * 16, dOs, LV);              // dA^T
-    uint32_t pa[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = e < 2 ? ka : kb, qi = nt * 8 + 2 * tg + (e & 1), query = q0 + qi;
-        const float a = (key <= query && query < T_) ? exp2f(fmaf(St[nt][e], c, -slse[qi])) : 0.f;
-        St[nt][e] = a;
-        dPt[nt][e] = a * (dPt[nt][e] - sD[qi]);              // dS^T
-      }
-    to_afrag(pa, St);
-    mm_kn<DV>(aV, pa, dOs, LV);                              // dV += A^T dO~
-    to_afrag(pa, dPt);
-    mm_kn<DQK>(aK, pa, Qs, LQ);                              // dK += dS^T Q
-  }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int key = e < 2 ? ka : kb;
-    if (key >= T_) continue;
-    const size_t rk = (size_t)b * T_ + key;
-#pragma unroll
-    for (int nt = 0; nt < DV / 8; ++nt) dV[(rk * H + h) * DV + nt * 8 + 2 * tg + (e & 1)] = aV[nt][e];
-#pragma unroll
-    for (int nt = 0; nt < DQK / 8; ++nt) {
-      const int col = nt * 8 + 2 * tg + (e & 1);
-      if (col < 128) dKC[(rk * H + h) * 128 + col] = aK[nt][e] * p.scale;
-      else atomicAdd(dkS + rk * 64 + (col - 128), aK[nt][e] * p.scale);
-    }
-  }
-}
-
-}  // namespace tc
 
 inline size_t workspace_bytes(int B, int T, int H, int d_v) {
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   return al((size_t)B * T * H * d_v * 4) + al((size_t)B * T * H * 4);
-}
-
-inline int run_tc(const Dims& p, const __nv_bfloat16* Q, const __nv_bfloat16* KC, const __nv_bfloat16* kS,
-                  const __nv_bfloat16* V, const __nv_bfloat16* g, const float* O, const float* lse, const float* dO,
-                  float* dQ, float* dKC, float* dkS, float* dV, float* dg, void* ws, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(tc::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM);
-    if (attr == cudaSuccess)
-      attr = cudaFuncSetAttribute(tc::dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::SMEM);
-  });
-  if (attr != cudaSuccess) return cuda_status(attr);
-  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  __nv_bfloat16* dOt = static_cast<__nv_bfloat16*>(ws);
-  float* D = reinterpret_cast<float*>(static_cast<char*>(ws) + al((size_t)p.B * p.T * p.H * p.d_v * 4));
-  const int rows = p.B * p.T * p.H;
-  cudaError_t e = cudaMemsetAsync(dkS, 0, (size_t)p.B * p.T * p.d_s * sizeof(float), st);
-  if (e != cudaSuccess) return cuda_status(e);
-  row_kernel<__nv_bfloat16, __nv_bfloat16><<<(rows + 7) / 8, 256, 0, st>>>(rows, p.H, p.d_v, O, dO, g, dOt, D, dg);
-  const int nt = (p.T + tc::R - 1) / tc::R;
-  tc::dkdv_kernel<<<dim3(nt, p.H, p.B), 128, tc::SMEM, st>>>(p, Q, KC, kS, V, lse, dOt, D, dKC, dkS, dV);
-  tc::dq_kernel<<<dim3(nt, p.H, p.B), 128, tc::SMEM, st>>>(p, Q, KC, kS, V, lse, dOt, D, dQ);
-  note_launches(3);
-  return check_launch();
 }
 
 template <typename T>

@@ -15,6 +15,7 @@
 #include "sm100.cuh"
 #include "tc_attn.cuh"
 #include "tc_decode.cuh"
+#include "tc_bwd.cuh"
 #include "tc_gemm.cuh"
 #include "attn_bwd.cuh"
 
@@ -76,14 +77,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 3-D bf16 tensor [d2][d1][d0] (d0 innermost, contiguous), box {64, 128, 1},
+// 3-D bf16 tensor [d2][d1][d0] (d0 innermost, contiguous), box {64, box1, 1},
 // 128-byte swizzle, out-of-range elements read as zero.
-static int make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2) {
+static int make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1 = 128) {
   auto enc = get_encode();
   if (!enc) return GMLA_EUNSUPPORTED;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -462,6 +463,53 @@ size_t mla_attn_bwd_workspace(const gmla_geom* g, int B, int T) {
   return bwd::workspace_bytes(B, T, g->H, g->d_v);
 }
 
+// Backward on the tcgen05 tensor cores (K3 head widths, bf16): the row pass
+// (dO~ in bf16 and D into the workspace), then the dK/dV and dQ kernels.
+static int attn_bwd_tc(const bwd::Dims& d, const __nv_bfloat16* Q, const __nv_bfloat16* KC,
+                       const __nv_bfloat16* kS, const __nv_bfloat16* V, const __nv_bfloat16* gate, const float* O,
+                       const float* lse, const float* dO, float* dQ, float* dKC, float* dkS, float* dV, float* dg,
+                       void* ws, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(tc_bwd::dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)tc_bwd::kv::SMEM_BYTES);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(tc_bwd::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tc_bwd::q::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  using bf = __nv_bfloat16;
+  const int B = d.B, T = d.T, H = d.H;
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  bf* dOt = static_cast<bf*>(ws);
+  float* D = reinterpret_cast<float*>(static_cast<char*>(ws) + al((size_t)B * T * H * 128 * 4));
+  // 64-row boxes for the tiles a CTA walks, 128-row boxes for its resident tile.
+  CUtensorMap mQ64, mDO64, mKC128, mKS128, mV128, mQ128, mDO128, mKC64, mKS64, mV64;
+  GMLA_TRY(make_map_3d(&mQ64, Q, (uint64_t)H * 192, T, B, 64));
+  GMLA_TRY(make_map_3d(&mDO64, dOt, (uint64_t)H * 128, T, B, 64));
+  GMLA_TRY(make_map_3d(&mKC128, KC, (uint64_t)H * 128, T, B, 128));
+  GMLA_TRY(make_map_3d(&mKS128, kS, 64, T, B, 128));
+  GMLA_TRY(make_map_3d(&mV128, V, (uint64_t)H * 128, T, B, 128));
+  GMLA_TRY(make_map_3d(&mQ128, Q, (uint64_t)H * 192, T, B, 128));
+  GMLA_TRY(make_map_3d(&mDO128, dOt, (uint64_t)H * 128, T, B, 128));
+  GMLA_TRY(make_map_3d(&mKC64, KC, (uint64_t)H * 128, T, B, 64));
+  GMLA_TRY(make_map_3d(&mKS64, kS, 64, T, B, 64));
+  GMLA_TRY(make_map_3d(&mV64, V, (uint64_t)H * 128, T, B, 64));
+  GMLA_TRY(cuda_status(cudaMemsetAsync(dkS, 0, (size_t)B * T * 64 * sizeof(float), st)));
+  const int rows = B * T * H;
+  bwd::row_kernel<bf, bf><<<(rows + 7) / 8, 256, 0, st>>>(rows, H, 128, O, dO, gate, dOt, D, dg);
+  tc_bwd::Params p;
+  p.B = B; p.T = T; p.H = H; p.lse = lse; p.D = D; p.dQ = dQ; p.dKC = dKC; p.dkS = dkS; p.dV = dV;
+  p.scale = d.scale;
+  p.scale_log2 = (float)(1.4426950408889634 * (double)d.scale);
+  const int nt = (T + 127) / 128;
+  tc_bwd::dkdv_kernel<<<dim3(nt, H, B), 192, tc_bwd::kv::SMEM_BYTES, st>>>(mQ64, mDO64, mKC128, mKS128, mV128, p);
+  tc_bwd::dq_kernel<<<dim3(nt, H, B), 192, tc_bwd::q::SMEM_BYTES, st>>>(mQ128, mDO128, mKC64, mKS64, mV64, p);
+  note_launches(3);
+  return check_launch();
+}
+
 int mla_attn_bwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void* Q, const void* KC, const void* kS,
                  const void* V, const void* gate, const float* O, const float* lse, const float* dO, float* dQ,
                  float* dKC, float* dkS, float* dV, float* dg, void* workspace, size_t workspace_bytes,
@@ -484,7 +532,7 @@ int mla_attn_bwd(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void*
                            (const float*)gate, O, lse, dO, dQ, dKC, dkS, dV, dg, workspace, st);
   using bf = __nv_bfloat16;
   if (is_k3_head_geometry(g))
-    return bwd::run_tc(p, (const bf*)Q, (const bf*)KC, (const bf*)kS, (const bf*)V, (const bf*)gate, O, lse, dO, dQ,
+    return attn_bwd_tc(p, (const bf*)Q, (const bf*)KC, (const bf*)kS, (const bf*)V, (const bf*)gate, O, lse, dO, dQ,
                        dKC, dkS, dV, dg, workspace, st);
   return bwd::run<bf>(p, (const bf*)Q, (const bf*)KC, (const bf*)kS, (const bf*)V, (const bf*)gate, O, lse, dO, dQ,
                       dKC, dkS, dV, dg, workspace, st);
