@@ -168,6 +168,10 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
           if (!wait_ok(RFULL + (i + 1) % NS, (uint32_t)((i + 1) / NS) & 1u)) break;
           // S^T buffer (i+1) & 1 held P^T(i-1), read by dV(i-1): issued earlier.
           issue_S(i + 1);
+          // dP^T's buffer is free once the compute warps have loaded dP^T(i)
+          // (they do that first), so dP^T(i+1) runs while they work on tile i.
+          if (!wait_ok(DPFREE, (uint32_t)i & 1u)) break;
+          issue_DP(i + 1);
         }
         if (!wait_ok(PFULL, (uint32_t)i & 1u)) break;
         const uint32_t q = slot_of(i);
@@ -182,11 +186,6 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                  sdesc_sw128(q + (uint32_t)kk * 2048u, SUB64, 1024), idDK, (i > 0 || kk > 0));
         mma_commit(bar(REMPTY + s));
         mma_commit(bar(DKDONE));
-        if (i + 1 < n_q) {
-          // dP^T's buffer is free once the softmax warps have loaded dP^T(i).
-          if (!wait_ok(DPFREE, (uint32_t)i & 1u)) break;
-          issue_DP(i + 1);
-        }
       }
       mma_commit(bar(DRAIN));
       mbar_wait_drain(bar(DRAIN), 0);
