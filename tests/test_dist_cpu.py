@@ -58,3 +58,39 @@ def test_maxlogit_allreduce_two_ranks():
     b = oracle.qkclip(WQ, WKV, ml_all.astype(np.float32), tau, geom, "f32")
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+def test_head_range_partitions_the_heads():
+    from gated_mla_qk_b200.dist import head_range
+    for H in (1, 4, 96, 97):
+        for world in (1, 2, 3, 5, 8):
+            ranges = [head_range(H, world, r) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == H
+            for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+                assert a1 == b0                      # contiguous, no overlap
+            sizes = [h1 - h0 for h0, h1 in ranges]
+            assert max(sizes) - min(sizes) <= 1      # balanced
+
+
+def test_head_sharded_clip_equals_full_clip_in_the_oracle():
+    """The clip of head h reads only maxlogit_h and writes only head h's columns, so
+    clipping each rank's contiguous column shard with its slice of the max-logit vector
+    and concatenating gives the full clip, bit for bit (the basis of head sharding)."""
+    from gated_mla_qk_b200.dist import head_range
+    geom = synth.Geom(H=7, d_model=32, q_lora=16, kv_lora=12, d_c=8, d_s=4, d_v=8)
+    rng = np.random.default_rng(3)
+    WQ = rng.standard_normal((geom.q_lora, geom.H * geom.d_qk)).astype(np.float32)
+    WKV = rng.standard_normal((geom.kv_lora, geom.H * (geom.d_c + geom.d_v))).astype(np.float32)
+    ml = np.array([3.0, 12.0, 9.0, 10.0, 50.0, -1.0, 10.5], np.float32)
+    full = oracle.qkclip(WQ, WKV, ml, 10.0, geom, "bf16")
+    w = geom.d_c + geom.d_v
+    for world in (2, 3, 7):
+        parts = []
+        for r in range(world):
+            h0, h1 = head_range(geom.H, world, r)
+            g = synth.Geom(H=h1 - h0, d_model=geom.d_model, q_lora=geom.q_lora, kv_lora=geom.kv_lora,
+                           d_c=geom.d_c, d_s=geom.d_s, d_v=geom.d_v)
+            parts.append(oracle.qkclip(WQ[:, h0 * geom.d_qk:h1 * geom.d_qk], WKV[:, h0 * w:h1 * w], ml[h0:h1], 10.0,
+                                       g, "bf16"))
+        for k, axis in ((0, 1), (1, 1), (2, 0), (3, 0)):
+            np.testing.assert_array_equal(np.concatenate([p[k] for p in parts], axis=axis), full[k])

@@ -32,7 +32,7 @@ def _train_and_backward(inp, geom, dO, gate):
     return host(lse), [host(x) if x is not None else None for x in (dQ, dKC, dkS, dV, dg)]
 
 
-@pytest.mark.parametrize("B,T,H,gate", [(1, 1, 2, True), (1, 70, 2, True), (2, 129, 3, False), (1, 300, 2, True),
+@pytest.mark.parametrize("B,T,H,gate", [(1, 1, 2, True), (1, 70, 2, True), (2, 129, 3, False), (1, 300, 2, True), (2, 520, 2, True),
                                          (1, 1000, 2, True)])
 def test_backward_k3_heads(B, T, H, gate):
     """K3 head widths (the tcgen05 training forward feeds o and lse)."""
