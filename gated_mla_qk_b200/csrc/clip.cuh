@@ -38,37 +38,61 @@ __device__ __forceinline__ void scale_vec(uint4& v, float f, float*) {
   for (int i = 0; i < 4; ++i) p[i] = __fmul_rn(p[i], f);
 }
 
-// Grid: x = blocks over (rows x vectors of the head's scaled columns),
-//       y = head, z = 0 for W_UQ, 1 for W_UKV.
+// Work items: (head h, matrix, chunk of kChunk 16-byte vectors of the head's
+// scaled columns), walked by a grid-stride loop, so the blocks of unclipped
+// heads cost one cached read of maxlogit[h] instead of a block launch each.
 // W_UQ : head block of d_c + d_s columns at h*(d_c+d_s): sqrt(gamma) then gamma.
 // W_UKV: head block at h*(d_c+d_v): the first d_c columns get sqrt(gamma).
+// Each thread loads its four vectors before scaling and storing them.
+constexpr int kPerThread = 4, kThreads = 256, kChunk = kPerThread * kThreads;
+
 template <typename T>
-__global__ void __launch_bounds__(256) qkclip_kernel(
+__global__ void __launch_bounds__(kThreads) qkclip_kernel(
     T* __restrict__ W_UQ, T* __restrict__ W_UKV, int q_lora, int kv_lora, int H, int d_c, int d_s,
     int d_v, const float* __restrict__ maxlogit, float tau, unsigned char* __restrict__ clipped,
     float* __restrict__ gamma_out) {
-  const int h = blockIdx.y;
-  float gam = 1.f, root = 1.f;
-  const bool clip = head_gamma(maxlogit, h, tau, &gam, &root);
-  if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
-    if (clipped) clipped[h] = clip ? 1 : 0;
-    if (gamma_out) gamma_out[h] = gam;
-  }
-  if (!clip) return;
   constexpr int VN = Vec<T>::n;
-  const bool is_q = blockIdx.z == 0;
-  const int cols = is_q ? (d_c + d_s) : d_c;              // scaled columns per row
-  const int rows = is_q ? q_lora : kv_lora;
-  const size_t ldw = is_q ? (size_t)H * (d_c + d_s) : (size_t)H * (d_c + d_v);
-  T* base = (is_q ? W_UQ : W_UKV) + (size_t)h * (is_q ? (d_c + d_s) : (d_c + d_v));
-  const int vpr = cols / VN;                               // vectors per row
-  const int total = rows * vpr;
-  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < total; v += gridDim.x * blockDim.x) {
-    const int r = v / vpr, c = (v - r * vpr) * VN;
-    uint4* p = reinterpret_cast<uint4*>(base + r * ldw + c);
-    uint4 x = *p;
-    scale_vec(x, c < d_c ? root : gam, (T*)nullptr);
-    *p = x;
+  if (blockIdx.x == 0)
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+      float gam = 1.f, root = 1.f;
+      const bool clip = head_gamma(maxlogit, h, tau, &gam, &root);
+      if (clipped) clipped[h] = clip ? 1 : 0;
+      if (gamma_out) gamma_out[h] = gam;
+    }
+  const int vq = q_lora * (d_c + d_s) / VN, vk = kv_lora * d_c / VN;   // vectors per head and matrix
+  const int nq = (vq + kChunk - 1) / kChunk, nk = (vk + kChunk - 1) / kChunk;
+  const int per_head = nq + nk;
+  for (int w = blockIdx.x; w < H * per_head; w += gridDim.x) {
+    const int h = w / per_head, k = w - h * per_head;
+    float gam = 1.f, root = 1.f;
+    if (!head_gamma(maxlogit, h, tau, &gam, &root)) continue;
+    const bool is_q = k < nq;
+    const int chunk = is_q ? k : k - nq;
+    const int cols = is_q ? (d_c + d_s) : d_c;              // scaled columns per row
+    const int total = is_q ? vq : vk;
+    const size_t ldw = is_q ? (size_t)H * (d_c + d_s) : (size_t)H * (d_c + d_v);
+    T* base = (is_q ? W_UQ : W_UKV) + (size_t)h * (is_q ? (d_c + d_s) : (d_c + d_v));
+    const int vpr = cols / VN;                               // vectors per row
+    uint4 x[kPerThread];
+    uint4* ptr[kPerThread];
+    float f[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int v = chunk * kChunk + u * kThreads + (int)threadIdx.x;
+      ptr[u] = nullptr;
+      if (v < total) {
+        const int r = v / vpr, c = (v - r * vpr) * VN;
+        ptr[u] = reinterpret_cast<uint4*>(base + r * ldw + c);
+        f[u] = c < d_c ? root : gam;
+        x[u] = *ptr[u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u)
+      if (ptr[u]) {
+        scale_vec(x[u], f[u], (T*)nullptr);
+        *ptr[u] = x[u];
+      }
   }
 }
 
@@ -102,13 +126,20 @@ inline int rescale(T* W_UQ, T* W_UKV, int q_lora, int kv_lora, int H, int d_c, i
                    const float* maxlogit, float tau, unsigned char* clipped, float* gamma, cudaStream_t st) {
   constexpr int VN = Vec<T>::n;
   const bool vec = (d_c % VN == 0) && (d_s % VN == 0) && (d_v % VN == 0);
-  const int per_head = max(q_lora * (d_c + d_s), kv_lora * d_c) / (vec ? VN : 1);
-  const int bx = min(64, max(1, (per_head + 255) / 256));
-  dim3 grid(bx, H, 2);
-  if (vec)
-    qkclip_kernel<T><<<grid, 256, 0, st>>>(W_UQ, W_UKV, q_lora, kv_lora, H, d_c, d_s, d_v, maxlogit, tau, clipped, gamma);
-  else
-    qkclip_scalar_kernel<T><<<grid, 256, 0, st>>>(W_UQ, W_UKV, q_lora, kv_lora, H, d_c, d_s, d_v, maxlogit, tau, clipped, gamma);
+  if (vec) {
+    const int items = H * ((q_lora * (d_c + d_s) / VN + kChunk - 1) / kChunk + (kv_lora * d_c / VN + kChunk - 1) / kChunk);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = max(1, min(items, 8 * sms));
+    qkclip_kernel<T><<<grid, kThreads, 0, st>>>(W_UQ, W_UKV, q_lora, kv_lora, H, d_c, d_s, d_v, maxlogit, tau,
+                                                clipped, gamma);
+  } else {
+    const int per_head = max(q_lora * (d_c + d_s), kv_lora * d_c);
+    const int bx = min(64, max(1, (per_head + 255) / 256));
+    qkclip_scalar_kernel<T><<<dim3(bx, H, 2), 256, 0, st>>>(W_UQ, W_UKV, q_lora, kv_lora, H, d_c, d_s, d_v, maxlogit,
+                                                            tau, clipped, gamma);
+  }
   note_launches(1);
   return check_launch();
 }
