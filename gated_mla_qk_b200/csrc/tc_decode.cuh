@@ -8,7 +8,7 @@
 //   q~_h = [q^C_h W_UK,h^T | q^S_h]                          (absorb kernel)
 //   s_j  = q~_h . cache_j / sqrt(192), p = softmax_j(s)
 //   u_h  = sum_j p_j cache_j[0:512]                          (split kernel)
-//   o_h  = (u_h / l) W_UV,h  (* sigmoid(g))                  (merge + project kernels)
+//   o_h  = (u_h / l) W_UV,h  (* sigmoid(g))                  (merge + projection kernel)
 //
 // Split kernel: a persistent grid of one CTA per SM.  The 96-token tiles of
 // all sequences, laid end to end, are cut into equal ranges, one per CTA, so
@@ -26,8 +26,8 @@
 // q~ (108 KB) stays in shared memory for the whole sequence.  The tile's
 // latent streams through a ring of three 24 KB slots twice: once, as 128-wide
 // latent pairs, for the score product, and once more (from L2, where the
-// first pass left it) for the value product after the softmax, so no slot is
-// held across the softmax and the ring stays short.  The 64 shared-key dims
+// first pass left it under an evict-last policy) for the value product after
+// the softmax, so no slot is held across the softmax and the ring stays short.  The 64 shared-key dims
 // have a slot of their own.  The score product of tile t+1 runs while the
 // softmax of tile t runs; S is released as soon as the softmax has loaded it.
 // Softmax: base-2 exponentials against a lazily updated reference max per
@@ -65,13 +65,9 @@ enum Bar { QFULL = 0, QEMPTY, LFULL, LEMPTY = LFULL + NPS, RFULL = LEMPTY + NPS,
            PVDONE, UFREE, DRAIN, NBAR };
 
 constexpr float kRescaleLog2 = 8.f;
-#ifndef GMLA_DEC_PF
-#define GMLA_DEC_PF 1
-#endif
-#ifndef GMLA_DEC_HINT
-#define GMLA_DEC_HINT 1
-#endif
-constexpr int kPrefetchAhead = GMLA_DEC_PF;   // tiles brought into L2 ahead of their first ring load
+// Tiles brought into L2 ahead of their first ring load.  One is enough; at
+// three the prefetched lines evicted the ones the second pass over a tile re-reads.
+constexpr int kPrefetchAhead = 1;
 
 struct SplitParams {
   int n_seq, G;
@@ -171,23 +167,17 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
       };
       int u = 0, seg = 0, rope_issued = 0;
       bool ok = true;
-#if GMLA_DEC_HINT
+      // The first pass over a tile keeps its lines in L2 for the second; the
+      // second pass is their last use.
       const uint64_t pol_keep = l2_policy_evict_last(), pol_drop = l2_policy_evict_first();
-#endif
       auto load_pair = [&](int row, int pr, bool second) {
         const uint32_t slot = (uint32_t)(u % NPS);
         if (!mbar_wait(bar(LEMPTY + slot), ((uint32_t)(u / NPS) & 1u) ^ 1u, abort)) { ok = false; return; }
         const uint32_t dst = sbase + OFF_PAIR + slot * PAIR;
         mbar_arrive_expect_tx(bar(LFULL + slot), PAIR);
-#if GMLA_DEC_HINT
         const uint64_t pol = second ? pol_drop : pol_keep;
         tma_load_2d_hint(dst, &tmC, bar(LFULL + slot), 128 * pr, row, pol);
         tma_load_2d_hint(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row, pol);
-#else
-        (void)second;
-        tma_load_2d(dst, &tmC, bar(LFULL + slot), 128 * pr, row);
-        tma_load_2d(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row);
-#endif
         ++u;
       };
       auto load_qk = [&](int t) {           // score-product items of tile t (cursor cq at t)
