@@ -177,7 +177,7 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   const uint64_t rows = std::min<uint64_t>((uint64_t)n * (uint64_t)max_len, 0x7fffffffull);
   GMLA_TRY(make_map_2d(&mC, cache, tc_dec::WID, rows, tc_dec::BT));
   GMLA_TRY(make_map_2d(&mQ, q_abs, tc_dec::WID, (uint64_t)n * tc_dec::HEADS, tc_dec::HEADS));
-  tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS, tc_dec::LAT / tc_dec::ABS_Q, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256,
+  tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS + 1, tc_dec::LAT / tc_dec::ABS_Q, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256,
                           tc_dec::ABS_SMEM, st>>>(
       n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs, offs, G, plan);
   tc_dec::SplitParams sp;

@@ -119,23 +119,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
 
-  // Launched behind the absorb kernel: q~ and the plan are its results.
-  griddep_wait();
-  griddep_launch_dependents();
-  int nt, i0, k0;
-  cta_range(p.plan, p.n_seq, p.G, cta, nt, i0, k0);
-  if (nt == 0) return;                                   // whole CTA: empty range
-  auto cursor = [&]() {
-    TileCursor cur;
-    cur.offs = p.offs; cur.n = p.n_seq; cur.k = k0;
-    cur.load(i0);
-    return cur;
-  };
-
   if (threadIdx.x == 0) abort_flag = device_error_pending() ? 1 : 0;
   __syncthreads();
   if (abort_flag) return;
   __syncthreads();
+  // Set-up that reads nothing of the absorb kernel's results, done while that
+  // kernel finishes (this grid is launched behind it).
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), (i == PFULL || i == UFREE || i == SFREE) ? 128 : 1);
     fence_mbar_init();
@@ -145,6 +134,21 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // q~ and the work plan are the absorb kernel's results.
+  griddep_wait();
+  griddep_launch_dependents();
+  int nt, i0, k0;
+  cta_range(p.plan, p.n_seq, p.G, cta, nt, i0, k0);
+  if (nt == 0) {                                         // whole CTA: empty range
+    if (warp == 5) tmem_dealloc(tmem, 512);
+    return;
+  }
+  auto cursor = [&]() {
+    TileCursor cur;
+    cur.offs = p.offs; cur.n = p.n_seq; cur.k = k0;
+    cur.load(i0);
+    return cur;
+  };
 
   // Ring order (producer and MMA thread walk it alike): the score-product
   // pairs of tile 0; then, per tile t, the score-product pairs of tile t+1
@@ -502,7 +506,7 @@ constexpr size_t ABS_SMEM = (size_t)(ABS_Q + ABS_SEQ) * LDK * 2;
 // columns, 64 sequences), 8 warps.  The block's rows of W_UK,h (128 x 128,
 // one 256-byte row segment per latent index) and its q^C rows are staged in
 // shared memory with 16-byte loads; warp w computes 16 latent columns.
-// Block (0, 0, 0) also builds the split kernel's work plan.
+// Block (HEADS, 0, 0) builds the split kernel's work plan meanwhile.
 __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ W_UKV,
                                                      __nv_bfloat16* __restrict__ q_abs, const int* __restrict__ offs,
@@ -514,7 +518,10 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   constexpr size_t ldw = (size_t)HEADS * 256;
   griddep_launch_dependents();                 // the split kernel may be scheduled (it waits for this grid)
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) build_plan(n_seq, offs, G, plan);
+  if (h == HEADS) {                            // the extra column of blocks: one of them builds the plan
+    if (blockIdx.y == 0 && blockIdx.z == 0) build_plan(n_seq, offs, G, plan);
+    return;
+  }
   for (int e = threadIdx.x; e < ABS_Q * 16; e += blockDim.x) {
     const int n = e >> 4, c = e & 15;
     cp_async16(Ws + n * LDK + c * 8, W_UKV + (size_t)(n0 + n) * ldw + (size_t)h * 256 + c * 8);
