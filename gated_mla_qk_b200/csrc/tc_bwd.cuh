@@ -234,18 +234,29 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         tc_fence_before();
         mbar_arrive(bar(DPFREE));
         uint32_t pk[32], dk[32];
+        // Query tiles from the third on lie wholly after the CTA's keys; only
+        // those that reach past T (and the first two) need the mask.
+        if (i >= 2 && q0 + 64 <= p.T) {
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int q = q0 + e + u;
-            const bool live = q < p.T && key <= q;  // causal: the key is at or before the query
-            pv[u] = live ? ex2(fmaf(s[e + u], c, -lse2[e + u])) : 0.f;
-            dv[u] = pv[u] * (dp[e + u] - Dq[e + u]);
+          for (int e = 0; e < 64; e += 2) {
+            const float p0 = ex2(fmaf(s[e], c, -lse2[e])), p1 = ex2(fmaf(s[e + 1], c, -lse2[e + 1]));
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+            dk[e >> 1] = pack_bf16x2(p0 * (dp[e] - Dq[e]), p1 * (dp[e + 1] - Dq[e + 1]));
           }
-          pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-          dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int q = q0 + e + u;
+              const bool live = q < p.T && key <= q;  // causal: the key is at or before the query
+              pv[u] = live ? ex2(fmaf(s[e + u], c, -lse2[e + u])) : 0.f;
+              dv[u] = pv[u] * (dp[e + u] - Dq[e + u]);
+            }
+            pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+            dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+          }
         }
         // P^T over the first 32 columns of its S^T buffer (read above).
         tmem_st32u(ts, pk);
@@ -460,16 +471,25 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&dp[32]));
       const int kb = 64 * j;
       uint32_t dk[32];
+      // Only the key tiles that reach past the tile's first row (and a row
+      // past T) need the mask.
+      if (kb + 63 <= q0 && valid) {
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        float dv[2];
+        for (int e = 0; e < 64; e += 2)
+          dk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], c, -lse2)) * (dp[e] - Dr),
+                                   ex2(fmaf(s[e + 1], c, -lse2)) * (dp[e + 1] - Dr));
+      } else {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const bool live = valid && kb + e + u <= t;   // causal (keys past T sit past every valid row)
-          const float pv = live ? ex2(fmaf(s[e + u], c, -lse2)) : 0.f;
-          dv[u] = pv * (dp[e + u] - Dr);
+        for (int e = 0; e < 64; e += 2) {
+          float dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const bool live = valid && kb + e + u <= t;   // causal (keys past T sit past every valid row)
+            const float pv = live ? ex2(fmaf(s[e + u], c, -lse2)) : 0.f;
+            dv[u] = pv * (dp[e + u] - Dr);
+          }
+          dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
         }
-        dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
       }
       // dS over the first 32 columns of its dP buffer (this thread's dP row is in registers).
       tmem_st32u(td, dk);
