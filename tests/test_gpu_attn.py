@@ -37,6 +37,7 @@ def _geom(H):
     (1, 300, 2, 1, False),     # ragged, no gate
     (2, 640, 4, 2, True),      # several tiles, several kv tiles per query tile
     (1, 1000, 3, 3, True),
+    (1, 300, 96, 8, True),     # every K3 head: the head-major grid and the max-logit atomics over 96 heads
 ])
 def test_small_against_full_oracle(B, T, H, hot, gate):
     geom = _geom(H)

@@ -33,7 +33,8 @@ def _train_and_backward(inp, geom, dO, gate):
 
 
 @pytest.mark.parametrize("B,T,H,gate", [(1, 1, 2, True), (1, 70, 2, True), (2, 129, 3, False), (1, 300, 2, True), (2, 520, 2, True),
-                                         (1, 1000, 2, True)])
+                                         (1, 1000, 2, True),
+                                         (1, 256, 96, True)])     # every K3 head: k^S's gradient summed over 96 heads
 def test_backward_k3_heads(B, T, H, gate):
     """K3 head widths (the tcgen05 training forward feeds o and lse)."""
     geom = synth.Geom(H=H)
