@@ -140,7 +140,10 @@ size_t mla_attn_bwd_workspace(const gmla_geom* geom, int B, int T);
  *   dQ [B][T][H][d_c+d_s], dKC [B][T][H][d_c], dkS [B][T][d_s],
  *   dV [B][T][H][d_v], dg [B][T][H*d_v] (required when g is given).
  * workspace: device scratch of at least mla_attn_bwd_workspace() bytes.
- * CUDA-core kernels, fp32 arithmetic; d_c+d_s <= 256, d_v <= 256.
+ * bf16 with d_c=128, d_s=64, d_v=128 runs the tcgen05/TMA kernels (A and dS
+ * enter the tensor-core products in bf16, accumulation in fp32); other shapes
+ * (d_c+d_s <= 256, d_v <= 256) and fp32 run CUDA-core kernels in fp32.
+ * dkS is zeroed on `stream` before the heads' contributions are added.
  */
 int mla_attn_bwd(const gmla_geom* geom, gmla_dtype dtype, int B, int T,
                  const void* Q, const void* KC, const void* kS, const void* V, const void* g,
