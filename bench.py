@@ -43,6 +43,17 @@ FWD_FLOP = 2.0 * B_FWD * 96 * T_FWD * (T_FWD + 1) / 2 * (192 + 128)
 T_TRAIN = 4096
 
 
+def workload_config(T_run, decode_tokens, parallelism):
+    """The `config` object of the JSON line; both arms print the same workload."""
+    return {"workload": "gated MLA attention fwd + maxlogit, B=1 T=16384 H=96 d_qk=192 d_v=128 bf16 "
+                        "(heads 0-7 x4); plus the K3 QK-Clip chain x[4,4096,7168] (up-proj, fwd, clip, "
+                        "recompute) and absorbed decode 64 seqs L~U[1024,8192] H=96",
+            "B": B_FWD, "T": T_run, "H": 96, "decode_tokens": decode_tokens,
+            "l2": "inputs larger than L2 (fwd inputs 1.8 GB, decode cache %.0f MB); no flush"
+                  % (decode_tokens * 576 * 2 / 1e6),
+            "parallelism": parallelism}
+
+
 def train_leg(args, gm, synth, geom, rank, st, dist):
     """mla_attn_fwd_train + mla_attn_bwd at B=1, T=4096, H=96 (gated, K3 heads)."""
     import torch
@@ -242,8 +253,10 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import numpy as np
     from gated_mla_qk_b200 import synth
     inp = synth.attn_core(B_FWD, T_FWD, synth.K3, seed=2, hot_heads=8, hot_scale=4.0)
+    decode_tokens = int(synth.decode_lengths(np.random.default_rng(4), 64, 1024, 8192).sum())
     for _ in range(args.warmup):
         oracle_sample(inp, rows_per_step=32)
     tot_s, tot_f = 0.0, 0.0
@@ -255,10 +268,10 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "attention core B=1 T=16384 H=96 (bounded sample per step: 32 heaviest rows of head 0)",
-                       "B": B_FWD, "T": T_FWD, "H": 96},
+            "config": workload_config(T_FWD, decode_tokens, "the oracle on rank 0's host cores"),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
-                             "sample": "per step: causal rows t=16352..16383 of head 0, float64 numpy"},
+                             "sample": "per step: the forward's 32 heaviest causal rows (t=16352..16383) of head 0 "
+                                       "at B=1, T=16384, float64 numpy; value = their causal FLOPs / time"},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -512,12 +525,8 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "gated MLA attention fwd + maxlogit, B=1 T=16384 H=96 d_qk=192 d_v=128 bf16 "
-                               "(heads 0-7 x4); plus the K3 QK-Clip chain x[4,4096,7168] (up-proj, fwd, clip, "
-                               "recompute) and absorbed decode 64 seqs L~U[1024,8192] H=96",
-                   "B": B_FWD, "T": T_run, "H": 96, "decode_tokens": total_tokens,
-                   "l2": "inputs larger than L2 (fwd inputs 1.8 GB, decode cache %.0f MB); no flush" % (dec_bytes_cache / 1e6),
-                   "parallelism": f"replicas x{world} (independent problems), maxlogit MAX all-reduce"},
+        "config": workload_config(T_run, total_tokens,
+                                  f"replicas x{world} (independent problems), maxlogit MAX all-reduce"),
         "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
                      "frac": fwd_tflops / pk["bf16"], "traffic": prof_traffic,
                      "kernel": "tc_attn::attn_fwd_kernel", "peak_source": f"{pk['src']} bf16 burst",

@@ -166,6 +166,11 @@ def k3_clip_layer(seed: int = 3, B: int = 4, T: int = 4096):
 # ---------------------------------------------------------------------------
 # Absorbed decode workload.
 # ---------------------------------------------------------------------------
+def decode_lengths(rng, n_seq: int, lo: int, hi: int) -> np.ndarray:
+    """Context lengths: integers U[lo, hi], the first draw of the decode workload's stream."""
+    return rng.integers(lo, hi + 1, size=n_seq).astype(np.int64)
+
+
 def decode_batch(n_seq: int = 64, lo: int = 1024, hi: int = 8192, geom: Geom = K3,
                  seed: int = 4, gate: bool = False, dtype: str = "bf16"):
     """64 sequences with integer context lengths U[lo, hi]; latent cache [sum L, 576] ~ N(0,1).
@@ -174,7 +179,7 @@ def decode_batch(n_seq: int = 64, lo: int = 1024, hi: int = 8192, geom: Geom = K
     belong to sequence i; each row is [c^KV (kv_lora) | k^S (d_s)].
     """
     rng = np.random.default_rng(seed)
-    lens = rng.integers(lo, hi + 1, size=n_seq).astype(np.int64)
+    lens = decode_lengths(rng, n_seq, lo, hi)
     offsets = np.zeros(n_seq + 1, np.int64)
     offsets[1:] = np.cumsum(lens)
     total = int(offsets[-1])
