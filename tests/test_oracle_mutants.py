@@ -24,12 +24,15 @@ from gated_mla_qk_b200 import synth
 
 def mutant(name, old, new, helper=None):
     """`name` from the oracle with `old` replaced by `new` in its source (or in
-    the source of `helper`, a function `name` calls)."""
+    the source of `helper`, a function `name` calls).  `old` and `new` may be
+    tuples of edits made together."""
     ns = dict(vars(M))
     target = helper or name
     src = inspect.getsource(getattr(M, target))
-    assert src.count(old) == 1, (target, old)
-    exec(compile(src.replace(old, new), f"<mutant of {target}>", "exec"), ns)
+    for o, n in (zip(old, new) if isinstance(old, tuple) else [(old, new)]):
+        assert src.count(o) == 1, (target, o)
+        src = src.replace(o, n)
+    exec(compile(src, f"<mutant of {target}>", "exec"), ns)
     if helper:                                     # re-bind `name` to the namespace that holds the mutated helper
         exec(compile(inspect.getsource(getattr(M, name)), f"<{name}>", "exec"), ns)
     return ns[name]
@@ -355,3 +358,90 @@ def test_rms_norm_mutant_is_caught(what):
 @pytest.mark.parametrize("what", sorted(UP_MUTANTS))
 def test_up_proj_mutant_is_caught(what):
     assert failing_pins([pin_up_proj_identity_layout], mutant(*UP_MUTANTS[what])), what
+
+
+# ---------------------------------------------------------------------------
+# row sampler, max-logit-only pass, log-sum-exp, materialised decode
+# ---------------------------------------------------------------------------
+def _sdpa_rows(Q, KC, kS, V, g, rows):
+    out = []
+    d_v = V.shape[-1]
+    for (b, t, h) in rows:
+        K = torch.cat([torch.from_numpy(KC[b, :t + 1, h]), torch.from_numpy(kS[b, :t + 1])], -1)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q[b, t, h])[None, None, None], K[None, None], torch.from_numpy(V[b, :t + 1, h])[None, None])
+        out.append(o[0, 0, 0].numpy() / (1 + np.exp(-g[b, t, h * d_v:(h + 1) * d_v])))
+    return np.stack(out)
+
+
+def pin_rows_vs_sdpa(impl):
+    Q, KC, kS, V, g = _attn_case()
+    rows = [(0, 0, 0), (1, 6, 1), (0, 3, 1), (1, 5, 0)]
+    got, _ = impl(Q, KC, kS, V, g, rows)
+    assert np.allclose(got, _sdpa_rows(Q, KC, kS, V, g, rows), rtol=1e-10, atol=1e-12)
+
+
+def pin_head_maxlogit_brute_force(impl):
+    Q, KC, kS, V, g = _attn_case()
+    got = impl(Q, KC, kS, heads=[0, 1])
+    pin_maxlogit_brute_force(lambda *a: (None, np.array([got[0], got[1]])))
+
+
+def pin_lse_vs_scipy(impl):
+    sp = pytest.importorskip("scipy.special")
+    Q, KC, kS, V, g = _attn_case()
+    lse = impl(Q, KC, kS)
+    B, T, H, d_qk = Q.shape
+    for b in range(B):
+        for h in range(H):
+            S = Q[b, :, h] @ np.concatenate([KC[b, :, h], kS[b]], -1).T / math.sqrt(d_qk)
+            for t in range(T):
+                assert lse[b, t, h] == pytest.approx(sp.logsumexp(S[t, :t + 1]), rel=1e-12)
+
+
+def pin_materialised_vs_sdpa(impl):
+    q, W, cache, offs, _ = _dec_case((9,), seed=28)
+    m = impl(q, W, cache, offs, G)
+    C, Wt = torch.from_numpy(cache), torch.from_numpy(W)
+    for h in range(G.H):
+        c0 = h * (G.d_c + G.d_v)
+        K = torch.cat([C[:, :G.kv_lora] @ Wt[:, c0:c0 + G.d_c], C[:, G.kv_lora:]], -1)
+        Vh = C[:, :G.kv_lora] @ Wt[:, c0 + G.d_c:c0 + G.d_c + G.d_v]
+        o = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[0, h])[None, None, None], K[None, None], Vh[None, None], scale=1.0 / math.sqrt(G.d_qk))
+        assert np.allclose(m[0, h], o[0, 0, 0].numpy(), rtol=1e-12, atol=1e-14)
+
+
+MISC = {
+    "row sample reads one key past the row": (pin_rows_vs_sdpa, (
+        "attention_rows", ("_f64(KC[b, :t + 1, h, :])", "_f64(kS[b, :t + 1])", "_f64(V[b, :t + 1, h, :])"),
+        ("_f64(KC[b, :t + 2, h, :])", "_f64(kS[b, :t + 2])", "_f64(V[b, :t + 2, h, :])"))),
+    "row sample queries from the previous position": (pin_rows_vs_sdpa, ("attention_rows", "q = _f64(Q[b, t, h, :])",
+                                                                         "q = _f64(Q[b, max(t - 1, 0), h, :])")),
+    "row sample gate of head 0": (pin_rows_vs_sdpa, ("attention_rows", "g[b, t, h * d_v:(h + 1) * d_v]", "g[b, t, :d_v]")),
+    "max-logit pass anti-causal": (pin_head_maxlogit_brute_force, ("head_maxlogit", "<= np.arange(t0, t1)[:, None]",
+                                                                   ">= np.arange(t0, t1)[:, None]")),
+    "max-logit pass unscaled": (pin_head_maxlogit_brute_force, ("head_maxlogit", "scale = 1.0 / math.sqrt(d_qk)", "scale = 1.0")),
+    "lse without the max": (pin_lse_vs_scipy, ("attention_lse", "(m + np.log(", "(0 * m + np.log(")),
+    "lse anti-causal": (pin_lse_vs_scipy, ("attention_lse", "causal = np.arange(T)[None, :] <= np.arange(T)[:, None]",
+                                           "causal = np.arange(T)[None, :] >= np.arange(T)[:, None]")),
+    "materialised 576-wide scale": (pin_materialised_vs_sdpa, ("decode_materialised", "scale = 1.0 / math.sqrt(geom.d_qk)",
+                                                               "scale = 1.0 / math.sqrt(geom.kv_lora + geom.d_s)")),
+    "materialised values from the K^C block": (pin_materialised_vs_sdpa, ("decode_materialised", "Vh = C[:, :geom.kv_lora] @ W_UV",
+                                                                          "Vh = C[:, :geom.kv_lora] @ W_UK[:, :geom.d_v]")),
+    "materialised keys without k^S": (pin_materialised_vs_sdpa, ("decode_materialised", "C[:, :geom.kv_lora] @ W_UK, C[:, geom.kv_lora:]",
+                                                                 "C[:, :geom.kv_lora] @ W_UK, 0 * C[:, geom.kv_lora:]")),
+}
+
+
+def test_misc_pins_pass_on_the_oracle():
+    assert failing_pins([pin_rows_vs_sdpa], oracle.attention_rows) == []
+    assert failing_pins([pin_head_maxlogit_brute_force], oracle.head_maxlogit) == []
+    assert failing_pins([pin_lse_vs_scipy], oracle.attention_lse) == []
+    assert failing_pins([pin_materialised_vs_sdpa], oracle.decode_materialised) == []
+
+
+@pytest.mark.parametrize("what", sorted(MISC))
+def test_misc_mutant_is_caught(what):
+    pin, spec = MISC[what]
+    assert failing_pins([pin], mutant(*spec)), what
