@@ -189,7 +189,9 @@ size_t mla_decode_workspace(const gmla_geom* geom, gmla_dtype dtype, int n_seq, 
  *   q [n_seq][H][d_c+d_s];  W_UKV [kv_lora][H*(d_c+d_v)]
  *   cache [total][kv_lora+d_s], sequence i = rows seq_offsets[i] .. seq_offsets[i+1]-1
  *   seq_offsets: device int32[n_seq+1], non-decreasing, seq_offsets[0] = 0,
- *     every length in [1, max_len]
+ *     every length in [1, max_len].  The offsets are device memory, so the host
+ *     does not check them; a zero or oversized length leaves every sequence's
+ *     output undefined (reads stay inside the cache rows the offsets name).
  *   g [n_seq][H*d_v] or NULL;  O [n_seq][H][d_v] (written)
  *   workspace: at least mla_decode_workspace() bytes.
  */
