@@ -61,6 +61,20 @@ static int check_dtype(gmla_dtype t) { return (t == GMLA_BF16 || t == GMLA_F32) 
 
 static inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// A kernel's dynamic shared-memory opt-in is an attribute of the kernel in
+// the current device's context, so it is set once per device the library is
+// called on (devices past the table are set on every call).
+constexpr int kMaxDevices = 64;
+template <typename F>
+static cudaError_t set_attributes_once(std::once_flag (&flags)[kMaxDevices], cudaError_t (&errs)[kMaxDevices], F set) {
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return set();
+  std::call_once(flags[dev], [&] { errs[dev] = set(); });
+  return errs[dev];
+}
+
 // ---------------------------------------------------------------------------
 // TMA descriptors (driver entry point fetched once through the runtime)
 // ---------------------------------------------------------------------------
@@ -140,19 +154,20 @@ static size_t decode_ws_bytes(const gmla_geom* g, gmla_dtype dtype, int n, int m
 
 static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache, const int* offs, int max_len,
                      const void* gate, void* O, void* ws, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc_dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)tc_dec::SMEM_BYTES);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(tc_dec::merge_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)tc_dec::MP_SMEM);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(tc_dec::absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)tc_dec::ABS_SMEM);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  const cudaError_t ae = set_attributes_once(once, attr_err, [] {
+    cudaError_t e = cudaFuncSetAttribute(tc_dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc_dec::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_dec::merge_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc_dec::MP_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_dec::absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc_dec::ABS_SMEM);
+    return e;
   });
-  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  if (ae != cudaSuccess) return cuda_status(ae);
   // One split CTA per SM (at most G_CAP), never more CTAs than tiles can exist.
   int dev = 0, sms = 0;
   GMLA_TRY(cuda_status(cudaGetDevice(&dev)));
@@ -206,16 +221,17 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
 static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const void* KC, const void* kS,
                        const void* V, const void* gate, void* O, bool out_f32, float* maxlogit, float* lse,
                        cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)tc_attn::SMEM_BYTES);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)tc_attn::SMEM_BYTES);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  const cudaError_t ae = set_attributes_once(once, attr_err, [] {
+    cudaError_t e = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc_attn::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_attn::attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc_attn::SMEM_BYTES);
+    return e;
   });
-  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  if (ae != cudaSuccess) return cuda_status(ae);
   CUtensorMap mQ, mKC, mKS, mV;
   const int H = g->H;
   GMLA_TRY(make_map_3d(&mQ, Q, (uint64_t)H * 192, T, B));
@@ -248,13 +264,13 @@ static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfl
     if (mode == 1) return simt::gemm<__nv_bfloat16>(M, N, K, A, B, simt::EpiSplitKV<__nv_bfloat16>{KC, V, H, d_c, d_v}, st);
     return simt::gemm<__nv_bfloat16>(M, N, K, A, B, simt::EpiPlain<__nv_bfloat16>{C, N}, st);
   }
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc_gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)tc_gemm::SMEM_BYTES);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  const cudaError_t ae = set_attributes_once(once, attr_err, [] {
+    return cudaFuncSetAttribute(tc_gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)tc_gemm::SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  if (ae != cudaSuccess) return cuda_status(ae);
   CUtensorMap mA, mB;
   GMLA_TRY(make_map_2d(&mA, A, (uint64_t)K, (uint64_t)M, tc_gemm::BM));
   GMLA_TRY(make_map_2d(&mB, B, (uint64_t)N, (uint64_t)K, tc_gemm::BK));
@@ -314,7 +330,6 @@ int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, c
 // ---------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;   // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-constexpr int kMaxDevices = 64;
 static std::mutex g_noalloc_mu;
 static void* g_noalloc_ptr[kMaxDevices] = {};
 
@@ -469,16 +484,17 @@ static int attn_bwd_tc(const bwd::Dims& d, const __nv_bfloat16* Q, const __nv_bf
                        const __nv_bfloat16* kS, const __nv_bfloat16* V, const __nv_bfloat16* gate, const float* O,
                        const float* lse, const float* dO, float* dQ, float* dKC, float* dkS, float* dV, float* dg,
                        void* ws, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc_bwd::dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)tc_bwd::kv::SMEM_BYTES);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(tc_bwd::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)tc_bwd::q::SMEM_BYTES);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t attr_err[kMaxDevices];
+  const cudaError_t ae = set_attributes_once(once, attr_err, [] {
+    cudaError_t e = cudaFuncSetAttribute(tc_bwd::dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc_bwd::kv::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_bwd::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc_bwd::q::SMEM_BYTES);
+    return e;
   });
-  if (attr_err != cudaSuccess) return cuda_status(attr_err);
+  if (ae != cudaSuccess) return cuda_status(ae);
   using bf = __nv_bfloat16;
   const int B = d.B, T = d.T, H = d.H;
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
