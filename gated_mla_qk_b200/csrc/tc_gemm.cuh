@@ -8,10 +8,11 @@
 // (64 x 256, N contiguous = MN-major) stream through a 4-stage TMA ring that
 // runs on across tile boundaries; one thread issues tcgen05.mma (M=128,
 // N=256, K=16) into one of two 256-column TMEM accumulators, so the four
-// epilogue warps read tile j back (tcgen05.ld, bf16 stores) while the MMAs
-// of tile j+1 run.  The epilogue either writes C row-major or, for the
-// key/value up-projection, splits each 256-column tile (= one head) into K^C
-// and V.
+// epilogue warps read tile j back (tcgen05.ld) while the MMAs of tile j+1
+// run.  Each epilogue warp stages 64-column chunks of its 32 rows in padded
+// shared memory and stores them as whole 128-byte lines.  The epilogue either
+// writes C row-major or, for the key/value up-projection, splits each
+// 256-column tile (= one head) into K^C and V.
 #pragma once
 
 #include "sm100.cuh"
