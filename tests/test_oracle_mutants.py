@@ -445,3 +445,95 @@ def test_misc_pins_pass_on_the_oracle():
 def test_misc_mutant_is_caught(what):
     pin, spec = MISC[what]
     assert failing_pins([pin], mutant(*spec)), what
+
+
+# ---------------------------------------------------------------------------
+# whole layer: the output gate g = x W_g and the output projection Delta = o W_O
+# ([OMA] "All 20 steps", output gate and output projection)
+# ---------------------------------------------------------------------------
+def _layer_case():
+    L = synth.tiny_layer(0)
+    return L, L["geom"]
+
+
+def _ungated_sdpa(L, geom):
+    """O~ (no gate) of the tiny layer from torch SDPA in float64 on the oracle's
+    up-projection outputs (the up-projection has its own pins above)."""
+    up = oracle.up_proj(L["x"], L["W_DQ"], L["w_q"], L["W_UQ"], L["W_DKV"], L["w_kv"], L["W_UKV"], geom, "f64")
+    B, T = L["x"].shape[:2]
+    out = np.empty((B, T, geom.H, geom.d_v))
+    for h in range(geom.H):
+        K = torch.cat([torch.from_numpy(up["KC"][:, :, h]), torch.from_numpy(up["kS"])], -1)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(up["Q"][:, :, h])[:, None], K[:, None], torch.from_numpy(up["V"][:, :, h])[:, None],
+            is_causal=True)[:, 0]
+        out[:, :, h] = o.numpy()
+    return out.reshape(B, T, -1)
+
+
+def pin_layer_zero_gate_halves_the_output(impl):
+    """W_g = 0 gives g = 0 and sigmoid(0) = 1/2 on every output column."""
+    L, geom = _layer_case()
+    L = dict(L, W_g=np.zeros_like(L["W_g"]))
+    res = impl(L["x"], L, geom, "f64")
+    assert np.allclose(res["o"], 0.5 * _ungated_sdpa(L, geom), rtol=1e-10, atol=1e-13)
+
+
+def pin_layer_gate_columns_line_up(impl):
+    """W_g[:, j] = c_j e_k: output column j is scaled by sigmoid(x_k c_j), c_j distinct per column."""
+    L, geom = _layer_case()
+    k = 5
+    c = np.linspace(-3.0, 3.0, geom.H * geom.d_v)
+    W_g = np.zeros_like(L["W_g"], dtype=np.float64)
+    W_g[k, :] = c
+    L = dict(L, W_g=W_g)
+    res = impl(L["x"], L, geom, "f64")
+    gate = torch.sigmoid(torch.from_numpy(L["x"][..., k:k + 1].astype(np.float64) * c)).numpy()
+    assert np.allclose(res["o"], gate * _ungated_sdpa(L, geom), rtol=1e-10, atol=1e-13)
+
+
+def pin_layer_output_projection_identity(impl):
+    """W_O = [I | 0] copies o into the first H d_v columns of Delta and leaves the rest 0;
+    a column permutation of it permutes Delta the same way."""
+    L, geom = _layer_case()
+    n = geom.H * geom.d_v
+    W_O = np.zeros((n, geom.d_model))
+    W_O[:, :n] = np.eye(n)
+    perm = np.random.default_rng(29).permutation(geom.d_model)
+    for W in (W_O, W_O[:, perm]):
+        res = impl(L["x"], dict(L, W_O=W), geom, "f64")
+        want = np.zeros(res["o"].shape[:2] + (geom.d_model,))
+        want[..., :n] = res["o"]
+        if W is not W_O:
+            want = want[..., perm]
+        assert np.array_equal(res["delta"], want)
+        assert np.allclose(res["o"], _layer_case_gated_reference(L, geom), rtol=1e-10, atol=1e-13)
+
+
+def _layer_case_gated_reference(L, geom):
+    gate = torch.sigmoid(torch.from_numpy(L["x"].astype(np.float64) @ L["W_g"].astype(np.float64))).numpy()
+    return gate * _ungated_sdpa(L, geom)
+
+
+LAYER_PINS = [pin_layer_zero_gate_halves_the_output, pin_layer_gate_columns_line_up, pin_layer_output_projection_identity]
+LAYER_MUTANTS = {
+    "gate dropped": ("layer_forward", 'up["V"], g)', 'up["V"], None)'),
+    "gate negated": ("layer_forward", 'up["V"], g)', 'up["V"], -g)'),
+    "gate read from W_O": ("layer_forward", 'g = _store(_f64(x) @ _f64(W["W_g"]), dtype)',
+                           'g = _store(_f64(x) @ _f64(W["W_O"]).T, dtype)'),
+    "gate columns reversed": ("layer_forward", 'g = _store(_f64(x) @ _f64(W["W_g"]), dtype)',
+                              'g = _store(_f64(x) @ _f64(W["W_g"])[:, ::-1], dtype)'),
+    "output projection from W_g": ("layer_forward", 'delta = o @ _f64(W["W_O"])', 'delta = o @ _f64(W["W_g"]).T'),
+    "output projection dropped": ("layer_forward", 'delta = o @ _f64(W["W_O"])', 'delta = _f64(x)'),
+    "o flattened feature-major": ("layer_forward", "o = _store(O.reshape(B, T, -1), dtype)",
+                                  "o = _store(O.transpose(0, 1, 3, 2).reshape(B, T, -1), dtype)"),
+}
+
+
+def test_layer_pins_pass_on_the_oracle():
+    assert failing_pins(LAYER_PINS, oracle.layer_forward) == []
+
+
+@pytest.mark.parametrize("what", sorted(LAYER_MUTANTS))
+def test_layer_mutant_is_caught(what):
+    assert failing_pins(LAYER_PINS, mutant(*LAYER_MUTANTS[what])), what
