@@ -454,48 +454,58 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const bool w = mbar_wait(bar(bi), ph, abort);
       return __all_sync(0xffffffffu, w) != 0;
     };
-    for (int j = 0; ok && j < n_k; ++j) {
+    // PFULL counts 128 arrivals per tile, and the S / dP of tile j+1 are
+    // usually ready before every warp has finished tile j.  A warp that ran a
+    // whole tile ahead would put its tile-(j+1) arrivals into tile j's phase,
+    // and the dQ product would read the dS rows of a warp that has not
+    // written them yet.  The vote at the end of each tile keeps the four warps
+    // in step (and makes a failed wait end the loop in all of them at once).
+    for (int j = 0; j < n_k; ++j) {
       const uint32_t par = (uint32_t)(j >> 1) & 1u;
-      if (!wait_warp(SFULL + (j & 1), par) || !wait_warp(DPFULL + (j & 1), par)) { ok = false; break; }
-      tc_fence_after();
-      float s[64], dp[64];
-      const uint32_t ts = tmem + lane_off + TS + 64u * (uint32_t)(j & 1);
-      const uint32_t td = tmem + lane_off + TDP + 64u * (uint32_t)(j & 1);
-      tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&s[0]));
-      tmem_ld32(ts + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
-      tmem_ld32(td, *reinterpret_cast<float(*)[32]>(&dp[0]));
-      tmem_ld32(td + 32u, *reinterpret_cast<float(*)[32]>(&dp[32]));
-      tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[0]));
-      tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[32]));
-      tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&dp[0]));
-      tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&dp[32]));
-      const int kb = 64 * j;
-      uint32_t dk[32];
-      // Only the key tiles that reach past the tile's first row (and a row
-      // past T) need the mask.
-      if (kb + 63 <= q0 && valid) {
+      if (ok) ok = wait_warp(SFULL + (j & 1), par) && wait_warp(DPFULL + (j & 1), par);
+      if (ok) {
+        tc_fence_after();
+        float s[64], dp[64];
+        const uint32_t ts = tmem + lane_off + TS + 64u * (uint32_t)(j & 1);
+        const uint32_t td = tmem + lane_off + TDP + 64u * (uint32_t)(j & 1);
+        tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_ld32(ts + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
+        tmem_ld32(td, *reinterpret_cast<float(*)[32]>(&dp[0]));
+        tmem_ld32(td + 32u, *reinterpret_cast<float(*)[32]>(&dp[32]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[32]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&dp[0]));
+        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&dp[32]));
+        const int kb = 64 * j;
+        uint32_t dk[32];
+        // Only the key tiles that reach past the tile's first row (and a row
+        // past T) need the mask.
+        if (kb + 63 <= q0 && valid) {
 #pragma unroll
-        for (int e = 0; e < 64; e += 2)
-          dk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], c, -lse2)) * (dp[e] - Dr),
-                                   ex2(fmaf(s[e + 1], c, -lse2)) * (dp[e + 1] - Dr));
-      } else {
+          for (int e = 0; e < 64; e += 2)
+            dk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], c, -lse2)) * (dp[e] - Dr),
+                                     ex2(fmaf(s[e + 1], c, -lse2)) * (dp[e + 1] - Dr));
+        } else {
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          float dv[2];
+          for (int e = 0; e < 64; e += 2) {
+            float dv[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const bool live = valid && kb + e + u <= t;   // causal (keys past T sit past every valid row)
-            const float pv = live ? ex2(fmaf(s[e + u], c, -lse2)) : 0.f;
-            dv[u] = pv * (dp[e + u] - Dr);
+            for (int u = 0; u < 2; ++u) {
+              const bool live = valid && kb + e + u <= t;   // causal (keys past T sit past every valid row)
+              const float pv = live ? ex2(fmaf(s[e + u], c, -lse2)) : 0.f;
+              dv[u] = pv * (dp[e + u] - Dr);
+            }
+            dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
           }
-          dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
         }
+        // dS over the first 32 columns of its dP buffer (this thread's dP row is in registers).
+        tmem_st32u(td, dk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(PFULL));
       }
-      // dS over the first 32 columns of its dP buffer (this thread's dP row is in registers).
-      tmem_st32u(td, dk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(PFULL));
+      ok = !bar_red_or(1, 128, !ok);
+      if (!ok) break;
     }
     if (ok) ok = wait_warp(DQDONE, 0);
     if (ok) {

@@ -34,3 +34,32 @@ def check_status():
     import gated_mla_qk_b200 as gm
     st = gm.device_status()
     assert st == 0, f"device status {st}"
+
+
+PAD = 4096          # guard bytes on each side; keeps the 16-byte (and 512-byte) alignment of the output
+
+
+class Guarded:
+    """A [PAD | nbytes | PAD] device buffer whose middle is viewed as ``shape`` of ``dtype``."""
+
+    def __init__(self, shape, dtype, init=None):
+        import torch
+        self.shape, self.dtype = tuple(shape), dtype
+        self.nbytes = int(np.prod(self.shape)) * torch.empty(0, dtype=dtype).element_size()
+        self.buf = torch.full((PAD + self.nbytes + PAD,), 0xFF, dtype=torch.uint8, device="cuda")
+        self.t = self.buf[PAD:PAD + self.nbytes].view(dtype).view(self.shape)
+        if init is not None:
+            self.t.copy_(init)
+
+    def check(self, name, written=True):
+        import torch
+        lo, hi = self.buf[:PAD], self.buf[PAD + self.nbytes:]
+        assert bool((lo == 0xFF).all()), f"{name}: bytes before the output were written"
+        assert bool((hi == 0xFF).all()), f"{name}: bytes after the output were written"
+        if written and self.dtype in (torch.float32, torch.bfloat16):
+            assert not bool(torch.isnan(self.t).any()), f"{name}: part of the output was never written"
+
+
+def guarded_bytes(n):
+    import torch
+    return Guarded((n,), torch.uint8)
