@@ -20,6 +20,17 @@ def max_rel(got, want) -> float:
     return float(np.max(np.abs(got - want) / np.abs(want)))
 
 
+def per_head(fn, heads, workers=8):
+    """Run the oracle one head at a time on a thread pool: fn(h) -> that head's
+    result.  numpy releases the GIL in its matrix products and elementwise
+    passes, so the heads of a long sequence overlap; each head's arithmetic is
+    the oracle's own, unchanged."""
+    from concurrent.futures import ThreadPoolExecutor
+    heads = list(heads)
+    with ThreadPoolExecutor(max(1, min(workers, len(heads)))) as ex:
+        return dict(zip(heads, ex.map(fn, heads)))
+
+
 def dev(a, dtype, device="cuda"):
     from gated_mla_qk_b200 import synth
     return None if a is None else synth.to_torch(a, dtype, device)

@@ -15,6 +15,7 @@ pytestmark = pytest.mark.gpu
     (1, 1536, 1536),       # a single row
     (300, 264, 520),       # ragged everything (N, K multiples of 8)
     (1024, 2048, 512),
+    (4096, 6144, 1536),    # 768 output tiles: every persistent CTA walks five or six, both TMEM accumulators cycle
 ])
 def test_gemm_bf16_vs_float64(M, N, K):
     import torch

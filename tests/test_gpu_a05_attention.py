@@ -1,14 +1,16 @@
 """Parity of mla_attn_fwd (bf16, K3 head geometry -> tcgen05 kernel) with the oracle.
 
-Small cases cover ragged and single-tile sequences against the full oracle;
-the two attention-core workloads (B=2,T=2048,H=96 and B=1,T=16384,H=96) are
-checked on sampled heads / rows and on the max logit of sampled heads."""
+Small cases cover ragged and single-tile sequences against the full oracle.
+The attention-core workload B=2, T=2048, H=96 is checked whole, head by head,
+with every head's max logit; the long-context workload B=1, T=16384, H=96 is
+checked on every head's max logit, on the whole output of 16 heads (heads
+0-7 and 8 seeded others) and on sampled rows of every head."""
 import numpy as np
 import pytest
 
 import oracle
 from gated_mla_qk_b200 import synth
-from gpu_util import TOL_BF16, TOL_MAXLOGIT, check_status, dev, host, max_rel, rel_l2
+from gpu_util import TOL_BF16, TOL_MAXLOGIT, check_status, dev, host, max_rel, per_head, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -79,31 +81,42 @@ def test_repeated_calls_identical():
 
 
 @pytest.mark.slow
-def test_core_T2048_sampled_heads():
-    """B=2, T=2048, H=96, heads 0-7 x3: full oracle on 6 heads, max logit on 16."""
+def test_core_T2048_every_head():
+    """B=2, T=2048, H=96, heads 0-7 x3: the whole output, head by head, and the
+    max logit of all 96 heads against the oracle."""
     inp = synth.attn_core_config("core_T2048")
     O, ml = _run(inp, synth.K3)
-    heads = [0, 3, 7, 8, 50, 95]
-    O_ref, _ = oracle.attention(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"], heads=heads)
-    assert rel_l2(O[:, :, heads], O_ref[:, :, heads]) <= TOL_BF16
-    ml_heads = list(range(8)) + [8, 20, 33, 47, 61, 70, 88, 95]
-    ref = oracle.head_maxlogit(inp["Q"], inp["KC"], inp["kS"], ml_heads)
-    got = ml[ml_heads]
-    want = np.array([ref[h] for h in ml_heads])
-    assert max_rel(got, want) <= TOL_MAXLOGIT
+    def one(h):                                    # keep only head h of the oracle's [B,T,H,d_v] result
+        O_ref, ml_ref = oracle.attention(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"], heads=[h])
+        return O_ref[:, :, h].copy(), ml_ref[h]
+    res = per_head(one, range(synth.K3.H))
+    for h, (O_h, ml_h) in res.items():
+        assert rel_l2(O[:, :, h], O_h) <= TOL_BF16, h
+        assert max_rel(ml[[h]], [ml_h]) <= TOL_MAXLOGIT, h
+    want = np.array([res[h][1] for h in range(synth.K3.H)])
     assert want[:8].min() > 2 * want[8:].max()     # the hot heads stand out
 
 
 @pytest.mark.slow
-def test_long_T16384_sampled_rows():
-    """B=1, T=16384, H=96, heads 0-7 x4: sampled rows one by one, max logit of 2 heads."""
+def test_long_T16384_heads_rows_and_every_max_logit():
+    """B=1, T=16384, H=96, heads 0-7 x4: the max logit of all 96 heads; the
+    whole output of heads 0-7 and of 8 seeded random heads at full T; and
+    sampled rows of every head."""
     inp = synth.attn_core_config("long_T16384")
     O, ml = _run(inp, synth.K3)
-    rng = np.random.default_rng(0)
-    rows = [(0, t, h) for h in (0, 5, 40, 95) for t in (0, 1, 127, 128, 4095, 8191, 12345, 16383)]
-    rows += [(0, int(t), int(h)) for t, h in zip(rng.integers(0, 16384, 16), rng.integers(0, 96, 16))]
-    want, _ = oracle.attention_rows(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"], rows)
+    H = synth.K3.H
+    ref = per_head(lambda h: oracle.head_maxlogit(inp["Q"], inp["KC"], inp["kS"], [h])[h], range(H))
+    want = np.array([ref[h] for h in range(H)])
+    assert max_rel(ml, want) <= TOL_MAXLOGIT
+    assert want[:8].min() > 2 * want[8:].max()
+    rng = np.random.default_rng(2)
+    heads = list(range(8)) + sorted(int(h) for h in rng.choice(np.arange(8, H), 8, replace=False))
+    full = per_head(lambda h: oracle.attention(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"], heads=[h])[0][:, :, h].copy(),
+                    heads, workers=4)
+    for h in heads:
+        assert rel_l2(O[:, :, h], full[h]) <= TOL_BF16, h
+    rows = [(0, t, h) for h in range(H) for t in (0, 127, 128, 8191, 16383)]
+    rows += [(0, int(t), int(h)) for t, h in zip(rng.integers(0, 16384, 96), rng.integers(0, H, 96))]
+    want_rows, _ = oracle.attention_rows(inp["Q"], inp["KC"], inp["kS"], inp["V"], inp["g"], rows)
     got = np.stack([O[b, t, h] for (b, t, h) in rows])
-    assert rel_l2(got, want) <= TOL_BF16
-    ref = oracle.head_maxlogit(inp["Q"], inp["KC"], inp["kS"], [0, 60])
-    assert max_rel(ml[[0, 60]], [ref[0], ref[60]]) <= TOL_MAXLOGIT
+    assert rel_l2(got, want_rows) <= TOL_BF16
