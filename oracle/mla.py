@@ -370,7 +370,9 @@ def decode_absorbed(q, W_UKV, cache, seq_offsets, geom, g=None):
       s_j  = q~_h . cache_j / sqrt(d_qk)            (the scale of the d_qk-wide head)
       u_h  = sum_j softmax(s)_j c^KV_j              (kv_lora)
       o_h  = u_h W_UV,h                             (d_v), then * sigmoid(g) if given.
-    Every cached token is visible (the query is the newest position).
+    Every cached token is visible (the query is the newest position).  A
+    sequence with no cached token has nothing to attend to; its output is the
+    empty sum, 0 (a reading: the pages never decode an empty cache).
     Returns O [n_seq, H, d_v] float64.
     """
     q, cache = _f64(q), _f64(cache)
@@ -383,6 +385,8 @@ def decode_absorbed(q, W_UKV, cache, seq_offsets, geom, g=None):
     O = np.zeros((n, H, geom.d_v))
     for i in range(n):
         C = cache[int(seq_offsets[i]):int(seq_offsets[i + 1])]          # [L, kv_lora + d_s]
+        if C.shape[0] == 0:
+            continue                                                      # empty cache: O[i] stays 0
         # q~_h = [q^C_h W_UK,h^T | q^S_h] for every head at once: [H, kv_lora + d_s]
         q_abs = np.concatenate([np.einsum("lhc,hc->hl", W_UK, q[i, :, :geom.d_c]), q[i, :, geom.d_c:]], axis=-1)
         s = (C @ q_abs.T) * scale                                         # [L, H]
@@ -401,6 +405,7 @@ def decode_materialised(q, W_UKV, cache, seq_offsets, geom, g=None):
     K_{h,j} = [c^KV_j W_UK,h | k^S_j], V_{h,j} = c^KV_j W_UV,h, then ordinary
     softmax attention of q_h over all cached positions ([FW] section 3: the
     training form materialises the per-head keys, decoding cannot afford to).
+    An empty cache gives 0, as in ``decode_absorbed``.
     """
     q, cache = _f64(q), _f64(cache)
     n = q.shape[0]
@@ -409,6 +414,8 @@ def decode_materialised(q, W_UKV, cache, seq_offsets, geom, g=None):
     O = np.zeros((n, H, geom.d_v))
     for i in range(n):
         C = cache[int(seq_offsets[i]):int(seq_offsets[i + 1])]
+        if C.shape[0] == 0:
+            continue
         for h in range(H):
             W_UK, W_UV = _uk_uv(W_UKV, geom, h)
             K = np.concatenate([C[:, :geom.kv_lora] @ W_UK, C[:, geom.kv_lora:]], axis=-1)

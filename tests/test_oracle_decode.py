@@ -80,3 +80,19 @@ def test_planted_mistake_wrong_scale_is_caught():
     scale_ratio = math.sqrt((G.kv_lora + G.d_s) / G.d_qk)
     b = oracle.decode_absorbed(q / scale_ratio, W, cache, offs, G)
     assert not np.allclose(a, b, rtol=1e-6)
+
+
+@pytest.mark.parametrize("fn", [oracle.decode_absorbed, oracle.decode_materialised])
+def test_empty_cache_gives_zero_and_leaves_the_others(fn):
+    """A sequence with no cached token decodes to 0 (the empty sum; the pages
+    never decode an empty cache), and dropping it changes no other sequence."""
+    lens = (0, 7, 0, 20, 0)
+    q, W, cache, offs, g = _case(lens=lens, seed=3, gate=True)
+    got = fn(q, W, cache, offs, G, g)
+    keep = [i for i, L in enumerate(lens) if L > 0]
+    for i, L in enumerate(lens):
+        if L == 0:
+            assert np.array_equal(got[i], np.zeros_like(got[i]))
+    offs2 = np.concatenate([[0], np.cumsum([lens[i] for i in keep])]).astype(np.int64)
+    want = fn(q[keep], W, cache, offs2, G, g[keep])
+    assert np.array_equal(got[keep], want)
