@@ -27,7 +27,7 @@ STATUS = {0: "GMLA_OK", -1: "GMLA_EINVAL", -2: "GMLA_EALIGN", -3: "GMLA_EUNSUPPO
           -5: "GMLA_ETIMEOUT", -6: "GMLA_EWORKSPACE"}
 
 EXPORTS = ["mla_up_proj_workspace", "mla_up_proj", "mla_attn_fwd", "mla_attn_fwd_train", "mla_attn_bwd_workspace", "mla_attn_bwd", "qkclip_rescale", "mla_decode_workspace",
-           "mla_decode_absorbed", "mla_decode_absorbed_noalloc", "mla_gemm", "gmla_device_status", "gmla_last_cuda_error", "gmla_strerror",
+           "mla_decode_absorbed", "mla_decode_absorbed_noalloc", "mla_gemm", "gmla_device_status", "gmla_set_wait_limit_ns", "gmla_selftest_wait", "gmla_last_cuda_error", "gmla_strerror",
            "gmla_version", "gmla_launch_count"]
 
 
@@ -78,6 +78,8 @@ def load_library(path: str = LIB_PATH):
         "mla_decode_absorbed_noalloc": (I, [G, I, I, P, P, P, P, I, P, P, P]),
         "mla_gemm": (I, [I, I, I, I, P, P, P, P]),
         "gmla_device_status": (I, [P]),
+        "gmla_set_wait_limit_ns": (I, [ctypes.c_ulonglong]),
+        "gmla_selftest_wait": (I, [P, P]),
         "gmla_last_cuda_error": (I, []),
         "gmla_strerror": (ctypes.c_char_p, [I]),
         "gmla_version": (I, []),
@@ -308,6 +310,18 @@ def mla_gemm(A, B, C, stream=None):
 def device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the library's device error status."""
     return load_library().gmla_device_status(_stream(stream))
+
+
+def set_wait_limit_ns(ns: int = 0) -> None:
+    """Limit of the kernels' device-side waits in nanoseconds (0: the 2 s default); see include/gmla.h."""
+    _check("gmla_set_wait_limit_ns", load_library().gmla_set_wait_limit_ns(int(ns)))
+
+
+def selftest_wait(elapsed, stream=None) -> None:
+    """Launch the bounded-wait self-test; ``elapsed`` is a CUDA int64 tensor of 2 (see include/gmla.h)."""
+    torch = _torch()
+    _check("gmla_selftest_wait", load_library().gmla_selftest_wait(_ptr(elapsed, "elapsed", torch.int64, 2),
+                                                                   _stream(stream)))
 
 
 def launch_count() -> int:

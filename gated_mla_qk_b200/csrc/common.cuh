@@ -48,10 +48,14 @@ __device__ __forceinline__ void raise_device_error(int code) {
   atomicCAS(&g_device_error, 0, code);
 }
 
-// Wall-time limit of every device-side wait (mbarrier try_wait loops).  Waits
+// Wall-time limit of the device-side waits (mbarrier try_wait loops).  Waits
 // inside one CTA normally last microseconds; one that lasts this long means
-// the pipeline is broken, and the kernel gives up instead of hanging.
+// the pipeline is broken, and the kernel gives up instead of hanging.  The
+// limit of the pipeline waits is a device variable (gmla_set_wait_limit_ns
+// shortens it, so that a test can make a wait run out); the drain waits a
+// giving-up CTA runs for its own copies and MMAs keep the fixed limit.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ bool device_error_pending() {
   return *reinterpret_cast<volatile int*>(&g_device_error) != 0;

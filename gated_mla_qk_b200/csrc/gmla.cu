@@ -18,6 +18,7 @@
 #include "tc_bwd.cuh"
 #include "tc_gemm.cuh"
 #include "attn_bwd.cuh"
+#include "selftest.cuh"
 
 namespace gmla {
 
@@ -375,6 +376,18 @@ const char* gmla_strerror(int s) {
     case GMLA_EWORKSPACE: return "workspace missing or too small";
     default: return "unknown status";
   }
+}
+
+int gmla_set_wait_limit_ns(unsigned long long ns) {
+  const uint64_t v = ns == 0 ? kWaitLimitNs : (uint64_t)ns;
+  return cuda_status(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+}
+
+int gmla_selftest_wait(unsigned long long* elapsed, void* stream) {
+  if (!elapsed) return GMLA_EINVAL;
+  selftest::wait_kernel<<<1, 64, 0, as_stream(stream)>>>(elapsed);
+  note_launches(1);
+  return check_launch();
 }
 
 int gmla_device_status(void* stream) {

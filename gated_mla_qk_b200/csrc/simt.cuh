@@ -374,7 +374,7 @@ __global__ void decode_combine_kernel(int H, int d_c, int d_v, int kv_lora, int 
   for (int s = 0; s < ns; ++s) M = fmaxf(M, part_ml[2 * (base + s)]);
   float Lsum = 0.f;
   for (int s = 0; s < ns; ++s) Lsum += part_ml[2 * (base + s) + 1] * expf(part_ml[2 * (base + s)] - M);
-  const float invL = 1.f / Lsum;
+  const float invL = Lsum > 0.f ? 1.f / Lsum : 0.f;   // an empty cache (no splits) decodes to 0
   for (int c = threadIdx.x; c < kv_lora; c += blockDim.x) {
     float u = 0.f;
     for (int s = 0; s < ns; ++s) u += part_u[(base + s) * kv_lora + c] * expf(part_ml[2 * (base + s)] - M);

@@ -59,7 +59,7 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Wait for the phase of parity `parity` to complete.  Gives up when *abort
 // is set by another warp of the CTA, when another CTA has already recorded a
-// device error, or after kWaitLimitNs of wall time; in the last case it
+// device error, or after g_wait_limit_ns of wall time; in the last case it
 // records GMLA_ETIMEOUT.  Giving up sets *abort and returns false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   uint64_t t0 = 0;
@@ -70,7 +70,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (device_error_pending()) { *abort = 1; return false; }
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) t0 = now;
-      else if (now - t0 > kWaitLimitNs) {
+      else if (now - t0 > g_wait_limit_ns) {
         raise_device_error(GMLA_ETIMEOUT);
         *abort = 1;
         return false;

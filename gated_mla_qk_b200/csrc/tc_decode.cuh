@@ -82,11 +82,13 @@ struct SplitParams {
 // Walks the tiles of a CTA's range: sequence i, tile k of it.  The tile's
 // BT-row window ends at the sequence's end when the tile is the last one, so
 // no row past the sequence (or the cache) is read; rows before the sequence
-// are masked (and rows before the cache read as zero).
+// are masked (and rows before the cache read as zero).  A sequence with an
+// empty cache has no tiles and is stepped over (the merge writes its zeros).
 struct TileCursor {
   const int* offs;
   int n, i, k, nti, L, start;
   __device__ void load(int seq) {
+    while (seq < n && offs[seq + 1] == offs[seq]) ++seq;
     i = seq;
     if (seq < n) { start = offs[seq]; L = offs[seq + 1] - start; nti = (L + BT - 1) / BT; }
   }

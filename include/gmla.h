@@ -189,9 +189,12 @@ size_t mla_decode_workspace(const gmla_geom* geom, gmla_dtype dtype, int n_seq, 
  *   q [n_seq][H][d_c+d_s];  W_UKV [kv_lora][H*(d_c+d_v)]
  *   cache [total][kv_lora+d_s], sequence i = rows seq_offsets[i] .. seq_offsets[i+1]-1
  *   seq_offsets: device int32[n_seq+1], non-decreasing, seq_offsets[0] = 0,
- *     every length in [1, max_len].  The offsets are device memory, so the host
- *     does not check them; a zero or oversized length leaves every sequence's
- *     output undefined (reads stay inside the cache rows the offsets name).
+ *     every length in [0, max_len].  A sequence of length 0 (an empty cache,
+ *     e.g. a free serving slot) gets an output row of zeros and does not
+ *     change any other sequence's output.  The offsets are device memory, so
+ *     the host does not check them; a length above max_len leaves every
+ *     sequence's output undefined (reads stay inside the cache rows the
+ *     offsets name).
  *   g [n_seq][H*d_v] or NULL;  O [n_seq][H][d_v] (written)
  *   workspace: at least mla_decode_workspace() bytes.
  */
@@ -210,11 +213,18 @@ int mla_decode_absorbed(const gmla_geom* geom, gmla_dtype dtype, int n_seq,
  * the same inputs and outputs as mla_decode_absorbed (minus the workspace) and
  * runs the same CUDA-core decode kernels on a scratch array that is part of
  * the library itself.
- *   Limit: the call needs at most mla_decode_workspace(geom, dtype, n_seq,
- *     max_len) bytes of scratch and the fixed array holds 16 MiB (16777216
- *     bytes); a request that needs more returns GMLA_EWORKSPACE and enqueues
- *     nothing.  Example: H=96, kv_lora=512 fits up to about 8 sequences of
- *     8192 tokens.
+ *   Limit: the fixed array holds 16 MiB (16777216 bytes).  This entry point
+ *     runs the CUDA-core decode kernels, whose scratch need is (with
+ *     S = ceil(max_len / 1024) splits per sequence and each of the first two
+ *     parts rounded up to a multiple of 256 bytes)
+ *       4 n_seq H (kv_lora + d_s)        absorbed queries
+ *     + 4 n_seq H S 2                    per-split (max, sum)
+ *     + 4 n_seq H S kv_lora              per-split latent sums
+ *     bytes (not mla_decode_workspace(), which sizes the tensor-core path).  A
+ *     request that needs more returns GMLA_EWORKSPACE and enqueues nothing.
+ *     Example: H = 96, kv_lora = 512, d_s = 64, max_len = 8192 needs
+ *     1,800,192 bytes per sequence, so 9 sequences fit (16,201,728 bytes) and
+ *     10 are refused.
  *   Memory: every GPU that loads the library holds the 16 MiB until the
  *     process exits.  No device memory is allocated by the call.
  *   Set-up: the first call on a device (the current device) looks up the
@@ -243,6 +253,29 @@ int mla_gemm(gmla_dtype dtype, int M, int N, int K, const void* A, const void* B
  * or GMLA_ETIMEOUT if a bounded device wait gave up since the last call.
  * GMLA_ECUDA if the synchronisation itself failed. */
 int gmla_device_status(void* stream);
+
+/* Wall-time limit, in nanoseconds, after which a device-side pipeline wait
+ * of this library's kernels gives up (default 2 s; 0 restores the default).
+ * The pages have no counterpart: this is the failure-detection hook.  A wait
+ * that gives up records GMLA_ETIMEOUT (read and cleared by
+ * gmla_device_status); its CTA stops issuing work, waits (with the fixed 2 s
+ * bound) for its own copies and MMAs still in flight, frees its tensor memory
+ * and returns, and CTAs that start afterwards return at once, so the context
+ * stays usable.  A short limit lets a test make a wait run out.  Applies to
+ * the current device, to kernels launched after the call; synchronous with
+ * respect to the host.  Do not change it while this library's kernels run. */
+int gmla_set_wait_limit_ns(unsigned long long ns);
+
+/* Self-test of the bounded waits: one CTA that holds tensor memory waits, as
+ * the pipeline kernels do, on an mbarrier that nothing ever arrives at.  The
+ * wait gives up after the current wait limit (gmla_set_wait_limit_ns) and
+ * records GMLA_ETIMEOUT; the CTA frees its tensor memory and returns.
+ * `elapsed` is a DEVICE pointer to two uint64: the wait's duration in ns and
+ * 1 if it gave up.  Asynchronous on `stream`; kernels of this library that
+ * start after it on the device return at once until gmla_device_status()
+ * has read the error.  The pages have no counterpart: this is the
+ * failure-detection test hook. */
+int gmla_selftest_wait(unsigned long long* elapsed, void* stream);
 
 /* The cudaError_t behind the last GMLA_ECUDA on this host thread (0 if none). */
 int gmla_last_cuda_error(void);

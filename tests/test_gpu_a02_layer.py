@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 from gated_mla_qk_b200 import synth
-from gpu_util import TOL_BF16, TOL_F32, TOL_MAXLOGIT, check_status, dev, host, max_rel, rel_l2
+from gpu_util import TOL_BF16, TOL_F32, check_status, dev, host, max_rel, rel_l2
 
 pytestmark = pytest.mark.gpu
 

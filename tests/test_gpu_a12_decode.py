@@ -19,7 +19,7 @@ def _run(d, dtype):
     O = torch.empty(n, geom.H, geom.d_v, dtype=td, device="cuda")
     offs = torch.from_numpy(d["seq_offsets"]).cuda()
     gm.mla_decode_absorbed(geom, dev(d["q"], dtype), dev(d["W_UKV"], dtype), dev(d["cache"], dtype), offs,
-                           int(d["lens"].max()), dev(d["g"], dtype), O)
+                           max(1, int(d["lens"].max())), dev(d["g"], dtype), O)
     check_status()
     return host(O)
 
@@ -96,3 +96,51 @@ def test_many_short_sequences():
     got = _run(d, "bf16")
     want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
     assert rel_l2(got, want) <= TOL_BF16
+
+
+@pytest.mark.parametrize("lens,gate", [((0, 5, 0, 0, 1000, 0, 129, 0), True), ((0,), False), ((0, 0, 0), True),
+                                       ((4096, 0), False)])
+def test_empty_caches_bf16(lens, gate):
+    """Sequences with an empty cache (a free serving slot) decode to rows of
+    zeros and leave every other sequence's output as the oracle has it."""
+    d = _with_lengths(lens, seed=45, gate=gate)
+    if d["cache"].shape[0] == 0:                  # no cached token at all: one row, never read
+        d["cache"] = np.zeros((1, 576), np.float32)
+    got = _run(d, "bf16")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
+    empty = np.array(lens) == 0
+    assert np.array_equal(got[empty], np.zeros_like(got[empty]))
+    if (~empty).any():
+        assert rel_l2(got[~empty], want[~empty]) <= TOL_BF16
+
+
+def test_many_short_sequences_with_empty_slots():
+    """160 sequences of 0-200 tokens, a third of them empty: ranges step over
+    the empty ones wherever they fall (first, last, in runs)."""
+    rng = np.random.default_rng(46)
+    lens = rng.integers(1, 201, size=160) * (rng.random(160) > 0.33)
+    lens[:3] = 0
+    lens[-2:] = 0
+    d = _with_lengths(tuple(int(x) for x in lens), seed=47, gate=True)
+    got = _run(d, "bf16")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], d["geom"], d["g"])
+    empty = lens == 0
+    assert np.array_equal(got[empty], np.zeros_like(got[empty]))
+    assert rel_l2(got[~empty], want[~empty]) <= TOL_BF16
+
+
+def test_empty_caches_fp32_tiny_geometry():
+    geom = synth.TINY
+    rng = np.random.default_rng(48)
+    lens = np.array([0, 5, 0, 300, 0])
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    n = len(lens)
+    d = dict(geom=geom, lens=lens, seq_offsets=offs,
+             cache=rng.standard_normal((int(offs[-1]), geom.kv_lora + geom.d_s)).astype(np.float32),
+             q=rng.standard_normal((n, geom.H, geom.d_qk)).astype(np.float32),
+             W_UKV=(rng.standard_normal((geom.kv_lora, geom.H * (geom.d_c + geom.d_v))) / 8).astype(np.float32),
+             g=rng.standard_normal((n, geom.H * geom.d_v)).astype(np.float32))
+    got = _run(d, "f32")
+    want = oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], geom, d["g"])
+    assert np.array_equal(got[lens == 0], np.zeros_like(got[lens == 0]))
+    assert rel_l2(got, want) <= TOL_F32

@@ -83,7 +83,8 @@ def test_qkclip_guards(dtype, geom):
     gamma.check("gamma")
 
 
-@pytest.mark.parametrize("lens,gate", [((1, 127, 1000, 129), True), ((5,), False), ((2048, 3, 4097), False)])
+@pytest.mark.parametrize("lens,gate", [((1, 127, 1000, 129), True), ((5,), False), ((2048, 3, 4097), False),
+                                       ((0, 127, 0, 1000, 0), True)])
 def test_decode_guards(lens, gate):
     import torch
     import gated_mla_qk_b200 as gm

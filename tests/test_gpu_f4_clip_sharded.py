@@ -15,7 +15,6 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("world", [2, 3, 5])
 def test_head_sharded_clip_matches_full_clip(world):
     import torch
-    import gated_mla_qk_b200 as gm
     from gated_mla_qk_b200.dist import head_range, qkclip_rescale_heads
     geom = synth.K3
     W = synth.layer_weights(geom, np.random.default_rng(40 + world), with_gate_out=False)

@@ -4,8 +4,9 @@ It exists for callers that cannot allocate device memory on their request
 path (a serving loop that must not call cudaMalloc/cudaFree, a plugin whose
 host owns all device memory).  The test calls it through the C ABI, twice in a
 row with different inputs, and checks each result against the workspace-taking
-entry point on the same inputs; it also checks that an oversized request is
-refused on the host.  This file sorts last so that a run stopping at the first
+entry point and against the oracle on the same inputs; at the size limit it
+checks that 9 sequences of 8192 tokens (16,201,728 bytes of scratch) run and
+match the oracle, and that 10 (18,001,920 bytes) are refused on the host.  This file sorts last so that a run stopping at the first
 failure has already run every other test.
 """
 import ctypes
@@ -13,6 +14,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 from gated_mla_qk_b200 import synth
 from gpu_util import TOL_BF16, rel_l2
 
@@ -57,6 +59,10 @@ def _with_workspace(d):
     return O.float().cpu().numpy()
 
 
+def _oracle(d):
+    return oracle.decode_absorbed(d["q"], d["W_UKV"], d["cache"], d["seq_offsets"], synth.K3, d["g"])
+
+
 def test_noalloc_decode_matches_workspace_decode_twice():
     import torch
     import gated_mla_qk_b200 as gm
@@ -65,18 +71,32 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     for seed, lens in ((41, (1, 300, 1024, 2047, 3000, 17)), (42, (2500, 5, 129, 128, 999, 2048))):
         d = _case(seed, lens)
         got = _noalloc_via_abi(lib, d, O)
-        want = _with_workspace(d)
-        assert rel_l2(got, want) <= TOL_BF16
+        assert rel_l2(got, _with_workspace(d)) <= TOL_BF16
+        assert rel_l2(got, _oracle(d)) <= TOL_BF16
 
 
-def test_noalloc_decode_refuses_oversized_request():
+def _scratch_need(n, max_len, H=96, kv_lora=512, d_s=64):
+    """The CUDA-core decode's scratch bytes, as include/gmla.h states them."""
+    al = lambda x: (x + 255) // 256 * 256
+    S = -(-max_len // 1024)
+    return al(4 * n * H * (kv_lora + d_s)) + al(4 * n * H * S * 2) + 4 * n * H * S * kv_lora
+
+
+def test_noalloc_decode_at_the_size_limit():
+    """9 sequences of 8192 tokens need 16,201,728 bytes of the 16 MiB scratch:
+    they run and match the oracle; 10 need 18,001,920 and are refused before
+    anything is enqueued."""
     import torch
     import gated_mla_qk_b200 as gm
     lib = gm.load_library()
     geom = gm.CGeom.of(synth.K3)
-    assert lib.mla_decode_workspace(ctypes.byref(geom), gm.GMLA_BF16, 64, 8192) > (16 << 20)
+    assert _scratch_need(9, 8192) == 16201728 <= (16 << 20) < _scratch_need(10, 8192) == 18001920
     p = torch.empty(16, dtype=torch.bfloat16, device="cuda").data_ptr()
     n0 = gm.launch_count()
-    st = lib.mla_decode_absorbed_noalloc(ctypes.byref(geom), gm.GMLA_BF16, 64, p, p, p, p, 8192, None, p, None)
+    st = lib.mla_decode_absorbed_noalloc(ctypes.byref(geom), gm.GMLA_BF16, 10, p, p, p, p, 8192, None, p, None)
     assert st == -6          # GMLA_EWORKSPACE, nothing enqueued
     assert gm.launch_count() == n0
+    d = _case(43, (8192,) * 9)
+    O = torch.empty(9, 96, 128, dtype=torch.bfloat16, device="cuda")
+    got = _noalloc_via_abi(lib, d, O)
+    assert rel_l2(got, _oracle(d)) <= TOL_BF16
