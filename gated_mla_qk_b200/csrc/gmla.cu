@@ -268,8 +268,12 @@ static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfl
   static std::once_flag once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
   const cudaError_t ae = set_attributes_once(once, attr_err, [] {
-    return cudaFuncSetAttribute(tc_gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)tc_gemm::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc_gemm::SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(tc_gemm::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tc_gemm::PAIR_SMEM_BYTES);
+    return e;
   });
   if (ae != cudaSuccess) return cuda_status(ae);
   CUtensorMap mA, mB;
@@ -277,13 +281,21 @@ static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfl
   GMLA_TRY(make_map_2d(&mB, B, (uint64_t)N, (uint64_t)K, tc_gemm::BK));
   tc_gemm::Params p;
   p.M = M; p.N = N; p.K = K; p.C = C; p.KC = KC; p.V = V; p.H = H; p.mode = mode;
-  // Persistent: one CTA per SM (never more CTAs than output tiles).
+  // Persistent: one CTA per SM (never more CTAs than output tiles); from 256
+  // rows on, CTA pairs on 256 x 256 tiles.
   int dev = 0, sms = 0;
   GMLA_TRY(cuda_status(cudaGetDevice(&dev)));
   GMLA_TRY(cuda_status(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)));
-  const long long tiles = (long long)((N + tc_gemm::BN - 1) / tc_gemm::BN) * ((M + tc_gemm::BM - 1) / tc_gemm::BM);
-  const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms));
-  tc_gemm::gemm_kernel<<<grid, 192, tc_gemm::SMEM_BYTES, st>>>(mA, mB, p);
+  const long long tiles_n = (N + tc_gemm::BN - 1) / tc_gemm::BN;
+  if (M >= tc_gemm::PAIR_BM) {
+    const long long tiles = tiles_n * ((M + tc_gemm::PAIR_BM - 1) / tc_gemm::PAIR_BM);
+    const unsigned pairs = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms / 2));
+    tc_gemm::gemm_pair_kernel<<<2 * pairs, 192, tc_gemm::PAIR_SMEM_BYTES, st>>>(mA, mB, p);
+  } else {
+    const long long tiles = tiles_n * ((M + tc_gemm::BM - 1) / tc_gemm::BM);
+    const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms));
+    tc_gemm::gemm_kernel<<<grid, 192, tc_gemm::SMEM_BYTES, st>>>(mA, mB, p);
+  }
   note_launches(1);
   return check_launch();
 }

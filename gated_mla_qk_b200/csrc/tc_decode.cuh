@@ -335,12 +335,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
       if (ok) {
         tc_fence_after();
         const uint32_t ts = tmem + lane_off + TM_S;
-        tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&s[0]));
-        tmem_ld32(ts + 32u, *reinterpret_cast<float(*)[32]>(&s[32]));
-        tmem_ld32(ts + 64u, *reinterpret_cast<float(*)[32]>(&s[64]));
-        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[0]));
-        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[32]));
-        tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[64]));
+        static_assert(BT % 32 == 0, "S is loaded in 32-column pieces");
+#pragma unroll
+        for (int k = 0; k < BT / 32; ++k) tmem_ld32(ts + 32u * k, *reinterpret_cast<float(*)[32]>(&s[32 * k]));
+#pragma unroll
+        for (int k = 0; k < BT / 32; ++k) tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&s[32 * k]));
         tc_fence_before();
         mbar_arrive(bar(SFREE));             // S may now be overwritten by the next tile's score product
         if (head) {
