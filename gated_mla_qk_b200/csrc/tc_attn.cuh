@@ -43,8 +43,10 @@ constexpr uint32_t OFF_RING = OFF_Q + 3 * SUB;
 constexpr uint32_t OFF_BAR = OFF_RING + NSTAGE * 3 * SUB;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;     // + barriers + alignment slack
 
+// P_j and the P.V product of tile j hand off through PFULL + (j & 1) and
+// PVDONE + (j & 1): a softmax warp may run one tile ahead of the MMA issuer.
 enum Bar { QFULL = 0, KVFULL = 1, KVEMPTY = KVFULL + NSTAGE, SFULL = KVEMPTY + NSTAGE, PFULL = SFULL + 2,
-           PVDONE = PFULL + 1, DRAIN = PVDONE + 1, NBAR = DRAIN + 1 };
+           PVDONE = PFULL + 2, DRAIN = PVDONE + 2, NBAR = DRAIN + 1 };
 
 constexpr float kRescaleLog2 = 8.f;   // rescale O when the row max grows by > 2^8
 
@@ -98,7 +100,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(bar(SFULL), 1);
     mbar_init(bar(SFULL + 1), 1);
     mbar_init(bar(PFULL), 128);
+    mbar_init(bar(PFULL + 1), 128);
     mbar_init(bar(PVDONE), 1);
+    mbar_init(bar(PVDONE + 1), 1);
     mbar_init(bar(DRAIN), 1);
     fence_mbar_init();
   }
@@ -180,7 +184,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           issue_S((j + 1) & 1, slot);
           ++u;
         }
-        if (!mbar_wait(bar(PFULL), (uint32_t)j & 1u, abort)) { ok = false; break; }
+        if (!mbar_wait(bar(PFULL + (j & 1)), (uint32_t)(j >> 1) & 1u, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t slot = u % NSTAGE, ph = (u / NSTAGE) & 1u;
         if (!mbar_wait(bar(KVFULL + slot), ph, abort)) { ok = false; break; }
@@ -193,7 +197,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint32_t vb = vbase + (uint32_t)i * 2048u;     // 16 keys x 128 B rows
           mma_ts(tO, tP + 8u * (uint32_t)i, sdesc_sw128(vb, SUB, 1024), idO, (j > 0 || i > 0));
         }
-        mma_commit(bar(PVDONE));
+        mma_commit(bar(PVDONE + (j & 1)));
         mma_commit(bar(KVEMPTY + slot));
         ++u;
       }
@@ -245,8 +249,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const bool need = (m_used == -INFINITY) || ((mx - m_used) * c > kRescaleLog2);
       const float m_new = need ? fmaxf(m_used, mx) : m_used;
       const float corr = need ? ex2((m_used - m_new) * c) : 1.f;
-      // Probabilities into registers first (bf16 pairs), so that they are
-      // computed while the P.V product of tile j-1 still reads the P buffer.
       const float neg = -m_new * c;
       uint32_t pk[64];
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -256,34 +258,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         ps[(e >> 1) & 7] += a0 + a1;
         pk[e >> 1] = pack_bf16x2(a0, a1);
       }
-      if (j > 0) {
-        if (!wait_warp(PVDONE, (uint32_t)(j - 1) & 1u)) { ok = false; break; }
+      // P_j goes over P_{j-2} in this S buffer, whose P.V product completed
+      // before S_j did (it was issued earlier).  Only a rescale of O waits,
+      // for the P.V product of tile j-1, which O must hold before it is scaled.
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if (!wait_warp(PVDONE + ((j - 1) & 1), (uint32_t)((j - 1) >> 1) & 1u)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float o[32];
-            tmem_ld32(tO_row + 32u * k, o);
-            tmem_wait_ld_dep(o);
+        for (int k = 0; k < 4; ++k) {
+          float o[32];
+          tmem_ld32(tO_row + 32u * k, o);
+          tmem_wait_ld_dep(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= corr;
-            tmem_st32(tO_row + 32u * k, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] *= corr;
+          tmem_st32(tO_row + 32u * k, o);
         }
+        tmem_wait_st();
       }
       l = l * corr + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
       m_used = m_new;
-      // P into TMEM over the first 64 columns of its own S buffer (S has been
-      // read; the score product that next writes this buffer is issued after
-      // this tile's P.V product).
+      // P into TMEM over the first 64 columns of its own S buffer.
       tmem_st32u(tS_row + (uint32_t)buf * 128u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
       tmem_st32u(tS_row + (uint32_t)buf * 128u + 32u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(PFULL));
+      mbar_arrive(bar(PFULL + buf));
     }
-    if (ok && wait_warp(PVDONE, (uint32_t)(n_kv - 1) & 1u)) {
+    if (ok && wait_warp(PVDONE + ((n_kv - 1) & 1), (uint32_t)((n_kv - 1) >> 1) & 1u)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool valid = t < p.T;
