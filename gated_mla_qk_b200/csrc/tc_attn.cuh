@@ -251,13 +251,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float corr = need ? ex2((m_used - m_new) * c) : 1.f;
       const float neg = -m_new * c;
       uint32_t pk[64];
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // Exponent arguments and row-sum partials two at a time (.f32x2).
+      const uint64_t c2 = f2(c, c), n2 = f2(neg, neg);
+      uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int e = 0; e < 128; e += 2) {
-        const float a0 = ex2(fmaf(s[e], c, neg)), a1 = ex2(fmaf(s[e + 1], c, neg));
-        ps[(e >> 1) & 7] += a0 + a1;
+        float x0, x1;
+        f2split(fma_f2(f2(s[e], s[e + 1]), c2, n2), x0, x1);
+        const float a0 = ex2(x0), a1 = ex2(x1);
+        ps2[(e >> 1) & 3] = add_f2(ps2[(e >> 1) & 3], f2(a0, a1));
         pk[e >> 1] = pack_bf16x2(a0, a1);
       }
+      float ps[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) f2split(ps2[q], ps[2 * q], ps[2 * q + 1]);
       // P_j goes over P_{j-2} in this S buffer, whose P.V product completed
       // before S_j did (it was issued earlier).  Only a rescale of O waits,
       // for the P.V product of tile j-1, which O must hold before it is scaled.

@@ -237,11 +237,17 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         // Query tiles from the third on lie wholly after the CTA's keys; only
         // those that reach past T (and the first two) need the mask.
         if (i >= 2 && q0 + 64 <= p.T) {
+          // Two scores at a time on the FMA pipe (.f32x2): exponent argument,
+          // dP - D and P (dP - D).
+          const uint64_t c2 = f2(c, c);
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
-            const float p0 = ex2(fmaf(s[e], c, -lse2[e])), p1 = ex2(fmaf(s[e + 1], c, -lse2[e + 1]));
+            float x0, x1, d0, d1;
+            f2split(fma_f2(f2(s[e], s[e + 1]), c2, f2(-lse2[e], -lse2[e + 1])), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
             pk[e >> 1] = pack_bf16x2(p0, p1);
-            dk[e >> 1] = pack_bf16x2(p0 * (dp[e] - Dq[e]), p1 * (dp[e + 1] - Dq[e + 1]));
+            f2split(mul_f2(f2(p0, p1), sub_f2(f2(dp[e], dp[e + 1]), f2(Dq[e], Dq[e + 1]))), d0, d1);
+            dk[e >> 1] = pack_bf16x2(d0, d1);
           }
         } else {
 #pragma unroll
@@ -481,10 +487,15 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         // Only the key tiles that reach past the tile's first row (and a row
         // past T) need the mask.
         if (kb + 63 <= q0 && valid) {
+          // Two scores at a time on the FMA pipe (.f32x2), as in dkdv_kernel.
+          const uint64_t c2 = f2(c, c), n2 = f2(-lse2, -lse2), D2 = f2(Dr, Dr);
 #pragma unroll
-          for (int e = 0; e < 64; e += 2)
-            dk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], c, -lse2)) * (dp[e] - Dr),
-                                     ex2(fmaf(s[e + 1], c, -lse2)) * (dp[e + 1] - Dr));
+          for (int e = 0; e < 64; e += 2) {
+            float x0, x1, d0, d1;
+            f2split(fma_f2(f2(s[e], s[e + 1]), c2, n2), x0, x1);
+            f2split(mul_f2(f2(ex2(x0), ex2(x1)), sub_f2(f2(dp[e], dp[e + 1]), D2)), d0, d1);
+            dk[e >> 1] = pack_bf16x2(d0, d1);
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
