@@ -122,6 +122,7 @@ def parse():
     ap.add_argument("--skip-decode", action="store_true", help="time the forward alone (profiling runs)")
     ap.add_argument("--skip-fwd", action="store_true", help="time the decode alone (profiling runs)")
     ap.add_argument("--skip-clip", action="store_true", help="leave out the K3 QK-Clip chain (profiling runs)")
+    ap.add_argument("--clip-T", type=int, default=4096, help="sequence length of the K3 QK-Clip chain (profiling runs)")
     ap.add_argument("--no-train", action="store_true", help="skip the training-form leg (fp32-output forward + backward)")
     return ap.parse_args()
 
@@ -322,7 +323,7 @@ def main():
     # ---- QK-Clip chain at K3 size ----
     chain = None
     if not args.skip_clip:
-        L = synth.k3_clip_layer(seed=3 + 1000 * rank)
+        L = synth.k3_clip_layer(seed=3 + 1000 * rank, T=args.clip_T)
         Bc, Tc = L["x"].shape[:2]
         bf = torch.bfloat16
         chain = dict(
@@ -336,8 +337,9 @@ def main():
         chain["WKV"] = chain["W"]["W_UKV"].clone()
         chain["ws"] = torch.empty(gm.mla_up_proj_workspace(geom, gm.GMLA_BF16, Bc, Tc), dtype=torch.uint8, device="cuda")
         del L
-    UP_FLOP = 2.0 * 4 * 4096 * (7168 * 1536 + 1536 * 18432 + 7168 * 576 + 512 * 24576)
-    C3_FLOP = 2.0 * 4 * 96 * 4096 * 4097 / 2 * 320
+    Mc = 4 * args.clip_T
+    UP_FLOP = 2.0 * Mc * (7168 * 1536 + 1536 * 18432 + 7168 * 576 + 512 * 24576)
+    C3_FLOP = 2.0 * 4 * 96 * args.clip_T * (args.clip_T + 1) / 2 * 320
 
     def clip_chain(ev):
         c = chain
@@ -547,10 +549,10 @@ def main():
         clip_ms = chain_sums[2] / args.steps
         clip_bytes = 2 * n_clipped * (1536 * 128 + 1536 * 64 + 512 * 128) * 2
         line["parts"] = {
-            "up_proj_B4_T4096": {"ms": up_ms, "value": UP_FLOP / (up_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "up_proj_B4_T%d" % args.clip_T: {"ms": up_ms, "value": UP_FLOP / (up_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                                  "roofline": {"bound": "tensor", "peak": pk["bf16"],
                                               "frac": UP_FLOP / (up_ms / 1e3) / 1e12 / pk["bf16"]}},
-            "attn_fwd_B4_T4096_nogate": {"ms": c3_ms, "value": C3_FLOP / (c3_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "attn_fwd_B4_T%d_nogate" % args.clip_T: {"ms": c3_ms, "value": C3_FLOP / (c3_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                                          "roofline": {"bound": "tensor", "peak": pk["bf16"],
                                                       "frac": C3_FLOP / (c3_ms / 1e3) / 1e12 / pk["bf16"]}},
             "qkclip": {"ms": clip_ms, "clipped_heads": n_clipped, "bytes": clip_bytes,
