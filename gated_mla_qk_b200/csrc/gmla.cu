@@ -319,11 +319,27 @@ int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, c
       return simt::gemm<T>(Mm, N, K, A, B, simt::EpiPlain<T>{C, N}, st);
   };
   GMLA_TRY(plain(M, g->q_lora, g->d_model, x, W_DQ, cQ));
-  simt::norm_rows_kernel<T><<<M, 256, 0, st>>>(cQ, g->q_lora, w_q, g->rms_eps, cQh);
+  // bf16 K3 widths: one warp per row (simt.cuh); otherwise one block per row.
+  constexpr bool bf = std::is_same<T, __nv_bfloat16>::value;
+  if constexpr (bf) {
+    if (g->q_lora == 1536)
+      simt::norm_rows_bf16_kernel<6><<<(M + 7) / 8, 256, 0, st>>>(cQ, M, w_q, g->rms_eps, cQh);
+    else
+      simt::norm_rows_kernel<T><<<M, 256, 0, st>>>(cQ, g->q_lora, w_q, g->rms_eps, cQh);
+  } else {
+    simt::norm_rows_kernel<T><<<M, 256, 0, st>>>(cQ, g->q_lora, w_q, g->rms_eps, cQh);
+  }
   note_launches(1);
   GMLA_TRY(plain(M, g->H * d_qk, g->q_lora, cQh, W_UQ, Q));
   GMLA_TRY(plain(M, g->kv_lora + g->d_s, g->d_model, x, W_DKV, ckv));
-  simt::norm_kv_rows_kernel<T><<<M, 256, 0, st>>>(ckv, g->kv_lora, g->d_s, w_kv, g->rms_eps, ckvh, kS, cache);
+  if constexpr (bf) {
+    if (g->kv_lora == 512 && g->d_s == 64)
+      simt::norm_kv_rows_bf16_kernel<2><<<(M + 7) / 8, 256, 0, st>>>(ckv, M, w_kv, g->rms_eps, ckvh, kS, cache);
+    else
+      simt::norm_kv_rows_kernel<T><<<M, 256, 0, st>>>(ckv, g->kv_lora, g->d_s, w_kv, g->rms_eps, ckvh, kS, cache);
+  } else {
+    simt::norm_kv_rows_kernel<T><<<M, 256, 0, st>>>(ckv, g->kv_lora, g->d_s, w_kv, g->rms_eps, ckvh, kS, cache);
+  }
   note_launches(1);
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
     GMLA_TRY(gemm_bf16(M, g->H * (g->d_c + g->d_v), g->kv_lora, ckvh, W_UKV, nullptr, KC, V, g->H, g->d_c, g->d_v, 1, st));

@@ -135,6 +135,101 @@ __global__ void norm_kv_rows_kernel(const T* __restrict__ ckv_ks, int kv_lora, i
   }
 }
 
+// bf16 forms of the two norms for row widths that are whole multiples of 256:
+// one warp per row, the row held in registers (NV 16-byte vectors per lane),
+// read once and written once with 16-byte accesses.
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __bfloat1622float2(h[e]);
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&f)[8]) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+  return u;
+}
+
+// out[m] = in[m] / sqrt(mean(in[m]^2) + eps) * w for n = 256 NV columns.
+template <int NV>
+__global__ void __launch_bounds__(256) norm_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in, int M,
+                                                             const __nv_bfloat16* __restrict__ w, float eps,
+                                                             __nv_bfloat16* __restrict__ out) {
+  constexpr int n = 256 * NV;
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (m >= M) return;
+  const uint4* src = reinterpret_cast<const uint4*>(in + (size_t)m * n);
+  float v[NV][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    unpack_bf16x8(src[lane + 32 * k], v[k]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(v[k][e], v[k][e], ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.f / sqrtf(ss / (float)n + eps);
+  uint4* dst = reinterpret_cast<uint4*>(out + (size_t)m * n);
+  const uint4* wv = reinterpret_cast<const uint4*>(w);
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    float wf[8], y[8];
+    unpack_bf16x8(wv[lane + 32 * k], wf);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = v[k][e] * inv * wf[e];
+    dst[lane + 32 * k] = pack_bf16x8(y);
+  }
+}
+
+// The key/value latent: a row of [c^KV (256 NV) | k^S (64)]; writes c^KV's
+// norm, k^S unchanged, and (if cache) the row [norm(c^KV) | k^S].
+template <int NV>
+__global__ void __launch_bounds__(256) norm_kv_rows_bf16_kernel(const __nv_bfloat16* __restrict__ ckv_ks, int M,
+                                                                const __nv_bfloat16* __restrict__ w, float eps,
+                                                                __nv_bfloat16* __restrict__ ckv_hat,
+                                                                __nv_bfloat16* __restrict__ kS,
+                                                                __nv_bfloat16* __restrict__ cache) {
+  constexpr int kv = 256 * NV, wid = kv + 64;
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (m >= M) return;
+  const uint4* src = reinterpret_cast<const uint4*>(ckv_ks + (size_t)m * wid);
+  float v[NV][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    unpack_bf16x8(src[lane + 32 * k], v[k]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(v[k][e], v[k][e], ss);
+  }
+  const uint4 ks = lane < 8 ? src[32 * NV + lane] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.f / sqrtf(ss / (float)kv + eps);
+  const uint4* wv = reinterpret_cast<const uint4*>(w);
+  uint4* hat = reinterpret_cast<uint4*>(ckv_hat + (size_t)m * kv);
+  uint4* crow = cache ? reinterpret_cast<uint4*>(cache + (size_t)m * wid) : nullptr;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    float wf[8], y[8];
+    unpack_bf16x8(wv[lane + 32 * k], wf);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = v[k][e] * inv * wf[e];
+    const uint4 u = pack_bf16x8(y);
+    hat[lane + 32 * k] = u;
+    if (crow) crow[lane + 32 * k] = u;
+  }
+  if (lane < 8) {
+    reinterpret_cast<uint4*>(kS + (size_t)m * 64)[lane] = ks;
+    if (crow) crow[32 * NV + lane] = ks;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Causal gated attention with the fused per-head max logit.
 // Block = (16 query rows, head h, batch b), 128 threads; key tiles of 32.
