@@ -110,6 +110,47 @@ def train_leg(args, gm, synth, geom, rank, st, dist):
     }
 
 
+def absorbed_leg(args, gm, synth, geom, rank, st, dist):
+    """mla_attn_fwd_absorbed (prefill on the latent cache) beside mla_attn_fwd at B=1, T=4096, H=96, gated."""
+    import torch
+    T, H = T_TRAIN, geom.H
+    gen = torch.Generator(device="cuda").manual_seed(7 + rank)
+    bf = torch.bfloat16
+    rnd = lambda *shape, s=1.0: (torch.randn(*shape, generator=gen, device="cuda") * s).to(bf)
+    Q, KC, kS, V = rnd(1, T, H, 192), rnd(1, T, H, 128), rnd(1, T, 64), rnd(1, T, H, 128)
+    cache, W, g = rnd(1, T, 576), rnd(512, H * 256, s=512 ** -0.5), rnd(1, T, H * 128)
+    O = torch.empty(1, T, H * 128, dtype=bf, device="cuda")
+    ml = torch.empty(H, dtype=torch.float32, device="cuda")
+    ws = torch.empty(gm.mla_attn_fwd_absorbed_workspace(geom, 1, T), dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(args.steps):
+            fn()
+        b.record(st)
+        torch.cuda.synchronize()
+        t = torch.tensor([a.elapsed_time(b) / args.steps], dtype=torch.float64, device="cuda")
+        if dist is not None:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    ms_abs = timed(lambda: gm.mla_attn_fwd_absorbed(geom, Q, W, cache, g, O, ml, ws))
+    ms_mat = timed(lambda: gm.mla_attn_fwd(geom, Q, KC, kS, V, g, O, ml))
+    pairs = H * T * (T + 1) / 2
+    return {"attn_fwd_absorbed_B1_T4096": {
+        "ms": ms_abs, "value": 2.0 * pairs * 320 / (ms_abs / 1e3) / 1e12, "unit": "TFLOP/s",
+        "own_work_tflops": 2.0 * pairs * (576 + 512) / (ms_abs / 1e3) / 1e12,
+        "materialised_fwd_ms": ms_mat,
+        "what": "mla_attn_fwd_absorbed: O and max logit from the latent cache (value counts the materialised "
+                "form's 320 MAC per pair, own_work_tflops the absorbed form's 1088)"}}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -500,6 +541,7 @@ def main():
     train = None
     if not args.no_train:
         train = train_leg(args, gm, synth, geom, rank, st, dist)
+        train.update(absorbed_leg(args, gm, synth, geom, rank, st, dist))
 
     if rank != 0:
         if dist is not None:

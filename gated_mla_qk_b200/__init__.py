@@ -27,7 +27,8 @@ STATUS = {0: "GMLA_OK", -1: "GMLA_EINVAL", -2: "GMLA_EALIGN", -3: "GMLA_EUNSUPPO
           -5: "GMLA_ETIMEOUT", -6: "GMLA_EWORKSPACE"}
 
 EXPORTS = ["mla_up_proj_workspace", "mla_up_proj", "mla_attn_fwd", "mla_attn_fwd_train", "mla_attn_bwd_workspace", "mla_attn_bwd", "qkclip_rescale", "mla_decode_workspace",
-           "mla_decode_absorbed", "mla_decode_absorbed_noalloc", "mla_gemm", "gmla_device_status", "gmla_set_wait_limit_ns", "gmla_selftest_wait", "gmla_last_cuda_error", "gmla_strerror",
+           "mla_decode_absorbed", "mla_decode_absorbed_noalloc", "mla_attn_fwd_absorbed_workspace",
+           "mla_attn_fwd_absorbed", "mla_gemm", "gmla_device_status", "gmla_set_wait_limit_ns", "gmla_selftest_wait", "gmla_last_cuda_error", "gmla_strerror",
            "gmla_version", "gmla_launch_count"]
 
 
@@ -76,6 +77,8 @@ def load_library(path: str = LIB_PATH):
         "mla_decode_workspace": (S, [G, I, I, I]),
         "mla_decode_absorbed": (I, [G, I, I, P, P, P, P, I, P, P, P, S, P]),
         "mla_decode_absorbed_noalloc": (I, [G, I, I, P, P, P, P, I, P, P, P]),
+        "mla_attn_fwd_absorbed_workspace": (S, [G, I, I]),
+        "mla_attn_fwd_absorbed": (I, [G, I, I, I, P, P, P, P, P, P, P, S, P]),
         "mla_gemm": (I, [I, I, I, I, P, P, P, P]),
         "gmla_device_status": (I, [P]),
         "gmla_set_wait_limit_ns": (I, [ctypes.c_ulonglong]),
@@ -293,6 +296,27 @@ def mla_decode_absorbed_noalloc(geom: Geom, q, W_UKV, cache, seq_offsets, max_le
         _ptr(W_UKV, "W_UKV", q.dtype, c["W_UKV"]), _ptr(cache, "cache", q.dtype),
         _ptr(seq_offsets, "seq_offsets", torch.int32, n + 1), int(max_len), _ptr(g, "g", q.dtype, c["O"]),
         _ptr(O, "O", q.dtype, c["O"]), _stream(stream)))
+
+
+def mla_attn_fwd_absorbed_workspace(geom: Geom, B: int, T: int) -> int:
+    return load_library().mla_attn_fwd_absorbed_workspace(ctypes.byref(CGeom.of(geom)), B, T)
+
+
+def mla_attn_fwd_absorbed(geom: Geom, Q, W_UKV, cache, g, O, maxlogit, workspace=None, stream=None):
+    """mla_attn_fwd's O and maxlogit computed on the latent cache (absorbed form); see include/gmla.h."""
+    lib = load_library()
+    torch = _torch()
+    _rank(Q, "Q", 4, "[B, T, H, d_c + d_s]")
+    B, T = Q.shape[0], Q.shape[1]
+    if workspace is None:
+        workspace = torch.empty(mla_attn_fwd_absorbed_workspace(geom, B, T), dtype=torch.uint8, device=Q.device)
+    n = _attn_counts(geom, B, T)
+    _check("mla_attn_fwd_absorbed", lib.mla_attn_fwd_absorbed(
+        ctypes.byref(CGeom.of(geom)), _dtype_code(Q), B, T, _ptr(Q, "Q", None, n["Q"]),
+        _ptr(W_UKV, "W_UKV", Q.dtype, geom.kv_lora * geom.H * (geom.d_c + geom.d_v)),
+        _ptr(cache, "cache", Q.dtype, B * T * (geom.kv_lora + geom.d_s)), _ptr(g, "g", Q.dtype, n["O"]),
+        _ptr(O, "O", Q.dtype, n["O"]), _ptr(maxlogit, "maxlogit", torch.float32, geom.H),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def mla_gemm(A, B, C, stream=None):

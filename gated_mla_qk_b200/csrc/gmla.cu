@@ -153,8 +153,13 @@ static size_t decode_ws_bytes(const gmla_geom* g, gmla_dtype dtype, int n, int m
   return b;
 }
 
-static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache, const int* offs, int max_len,
-                     const void* gate, void* O, void* ws, cudaStream_t st) {
+// Absorbed attention of n queries over windows of the latent cache (decode:
+// one window per sequence; prefill: each query's causal prefix).  cache_rows
+// bounds the cache rows any window reaches, max_tiles the 96-token tiles of
+// all windows; maxlogit (nullable) gets the per-head max of the scaled logits.
+static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache, tc_dec::Windows win,
+                     uint64_t cache_rows, long long max_tiles, const void* gate, void* O, float* maxlogit, void* ws,
+                     cudaStream_t st) {
   static std::once_flag once[kMaxDevices];
   static cudaError_t attr_err[kMaxDevices];
   const cudaError_t ae = set_attributes_once(once, attr_err, [] {
@@ -173,7 +178,6 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   int dev = 0, sms = 0;
   GMLA_TRY(cuda_status(cudaGetDevice(&dev)));
   GMLA_TRY(cuda_status(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)));
-  const long long max_tiles = (long long)n * ((max_len + tc_dec::BT - 1) / tc_dec::BT);
   const int G = (int)std::max<long long>(1, std::min<long long>(std::min(sms, tc_dec::G_CAP), max_tiles));
   using bf = __nv_bfloat16;
   auto al = [](size_t x) { return (x + 1023) & ~(size_t)1023; };
@@ -187,19 +191,21 @@ static int decode_tc(int n, const void* q, const void* W_UKV, const void* cache,
   p += al(np * tc_dec::HEADS * 2 * 4);
   float* part_u = reinterpret_cast<float*>(p);
   CUtensorMap mC, mQ;
-  // Rows of the cache map: every row a tile reads lies inside some sequence
-  // (the last tile of a sequence is shifted back to end at its end), so
-  // n * max_len bounds the coordinates that occur; rows before 0 read as zero.
-  const uint64_t rows = std::min<uint64_t>((uint64_t)n * (uint64_t)max_len, 0x7fffffffull);
+  // Rows of the cache map: every row a tile reads lies inside some window
+  // (the last tile of a window is shifted back to end at its end), so
+  // cache_rows bounds the coordinates that occur; rows before 0 read as zero.
+  const uint64_t rows = std::min<uint64_t>(cache_rows, 0x7fffffffull);
   GMLA_TRY(make_map_2d(&mC, cache, tc_dec::WID, rows, tc_dec::BT));
   GMLA_TRY(make_map_2d(&mQ, q_abs, tc_dec::WID, (uint64_t)n * tc_dec::HEADS, tc_dec::HEADS));
   tc_dec::absorb_kernel<<<dim3(tc_dec::HEADS + 1, tc_dec::LAT / tc_dec::ABS_Q, (n + tc_dec::ABS_SEQ - 1) / tc_dec::ABS_SEQ), 256,
                           tc_dec::ABS_SMEM, st>>>(
-      n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs, offs, G, plan);
+      n, static_cast<const bf*>(q), static_cast<const bf*>(W_UKV), q_abs, win, G, plan);
   tc_dec::SplitParams sp;
-  sp.n_seq = n; sp.G = G; sp.offs = offs; sp.plan = plan; sp.cache = static_cast<const bf*>(cache);
+  sp.n_seq = n; sp.G = G; sp.win = win; sp.plan = plan; sp.cache = static_cast<const bf*>(cache);
   sp.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   sp.part_ml = part_ml; sp.part_u = part_u;
+  sp.maxlogit = maxlogit;
+  sp.scale = 1.f / std::sqrt(192.f);
   // The split and merge kernels are launched behind their predecessor
   // (programmatic dependent launch): each waits for it with griddepcontrol.wait
   // before touching its results, so only their set-up overlaps its tail.
@@ -632,7 +638,8 @@ int mla_decode_absorbed(const gmla_geom* g, gmla_dtype dtype, int n_seq, const v
   if (!aligned16(workspace)) return GMLA_EALIGN;
   cudaStream_t st = as_stream(stream);
   if (dtype == GMLA_BF16 && is_k3_decode_geometry(g))
-    return decode_tc(n_seq, q, W_UKV, cache, seq_offsets, max_len, gate, O, workspace, st);
+    return decode_tc(n_seq, q, W_UKV, cache, tc_dec::Windows{seq_offsets, 0}, (uint64_t)n_seq * (uint64_t)max_len,
+                     (long long)n_seq * ((max_len + tc_dec::BT - 1) / tc_dec::BT), gate, O, nullptr, workspace, st);
   if (dtype == GMLA_F32)
     return simt::decode<float>(n_seq, g->H, g->d_c, g->d_s, g->d_v, g->kv_lora, (const float*)q,
                                (const float*)W_UKV, (const float*)cache, seq_offsets, max_len, (const float*)gate,
@@ -640,6 +647,39 @@ int mla_decode_absorbed(const gmla_geom* g, gmla_dtype dtype, int n_seq, const v
   using bf = __nv_bfloat16;
   return simt::decode<bf>(n_seq, g->H, g->d_c, g->d_s, g->d_v, g->kv_lora, (const bf*)q, (const bf*)W_UKV,
                           (const bf*)cache, seq_offsets, max_len, (const bf*)gate, (bf*)O, workspace, st);
+}
+
+// ---------------------------------------------------------------------------
+// Prefill on the latent cache: mla_attn_fwd's outputs computed the absorbed
+// way, each query over its causal prefix of the cache.
+size_t mla_attn_fwd_absorbed_workspace(const gmla_geom* g, int B, int T) {
+  if (check_geom(g) != GMLA_OK || !is_k3_decode_geometry(g) || B <= 0 || T <= 0) return 0;
+  if ((long long)B * T > (1LL << 24)) return 0;
+  return tc_dec::workspace_bytes(B * T);
+}
+
+int mla_attn_fwd_absorbed(const gmla_geom* g, gmla_dtype dtype, int B, int T, const void* Q, const void* W_UKV,
+                          const void* cache, const void* gate, void* O, float* maxlogit, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  GMLA_TRY(check_geom(g));
+  GMLA_TRY(check_dtype(dtype));
+  if (B <= 0 || T <= 0) return GMLA_EINVAL;
+  GMLA_REQUIRE(Q); GMLA_REQUIRE(W_UKV); GMLA_REQUIRE(cache); GMLA_REQUIRE(O); GMLA_REQUIRE(maxlogit);
+  GMLA_OPTIONAL(gate);
+  if (dtype != GMLA_BF16 || !is_k3_decode_geometry(g)) return GMLA_EUNSUPPORTED;
+  if ((long long)B * T > (1LL << 24)) return GMLA_EUNSUPPORTED;
+  if (!workspace || workspace_bytes < mla_attn_fwd_absorbed_workspace(g, B, T)) return GMLA_EWORKSPACE;
+  if (!aligned16(workspace)) return GMLA_EALIGN;
+  cudaStream_t st = as_stream(stream);
+  const int n = B * T;
+  // Query b*T + t reads rows b*T .. b*T + t: ceil((t+1) / 96) tiles each.
+  long long tiles = 0;
+  for (int t = 0; t < T; ++t) tiles += (t + tc_dec::BT) / tc_dec::BT;
+  simt::fill_kernel<<<(g->H + 127) / 128, 128, 0, st>>>(maxlogit, g->H, -INFINITY);
+  note_launches(1);
+  GMLA_TRY(check_launch());
+  return decode_tc(n, Q, W_UKV, cache, tc_dec::Windows{nullptr, T}, (uint64_t)n, tiles * B, gate, O, maxlogit,
+                   workspace, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -69,14 +69,27 @@ constexpr float kRescaleLog2 = 8.f;
 // three the prefetched lines evicted the ones the second pass over a tile re-reads.
 constexpr int kPrefetchAhead = 1;
 
+// The cache rows each query attends to.  Decode: sequence i owns the packed
+// rows offs[i] .. offs[i+1]-1.  Prefill on the latent cache (prefix_T > 0):
+// query i = b * prefix_T + t attends to rows b * prefix_T .. b * prefix_T + t,
+// its own causal prefix.
+struct Windows {
+  const int* offs;                 // [n_seq + 1] (decode)
+  int prefix_T;                    // > 0: prefill, sequence length
+  __device__ int start(int i) const { return prefix_T > 0 ? (i / prefix_T) * prefix_T : offs[i]; }
+  __device__ int len(int i) const { return prefix_T > 0 ? i % prefix_T + 1 : offs[i + 1] - offs[i]; }
+};
+
 struct SplitParams {
   int n_seq, G;
-  const int* offs;                 // [n_seq + 1]
+  Windows win;
   const __nv_bfloat16* cache;      // [rows][576]
   const int* plan;                 // [n_seq + 1] tile prefix, then [G] first sequence of each CTA
   float scale_log2;                // log2(e) / sqrt(192)
   float* part_ml;                  // [G + n_seq][96][2]: reference max (raw logit units), sum
   float* part_u;                   // [G + n_seq][96][512]
+  float* maxlogit;                 // [96] or nullptr: per-head max of the scaled logits (atomic max)
+  float scale;                     // 1 / sqrt(192)
 };
 
 // Walks the tiles of a CTA's range: sequence i, tile k of it.  The tile's
@@ -85,12 +98,12 @@ struct SplitParams {
 // are masked (and rows before the cache read as zero).  A sequence with an
 // empty cache has no tiles and is stepped over (the merge writes its zeros).
 struct TileCursor {
-  const int* offs;
+  Windows win;
   int n, i, k, nti, L, start;
   __device__ void load(int seq) {
-    while (seq < n && offs[seq + 1] == offs[seq]) ++seq;
+    while (seq < n && win.len(seq) == 0) ++seq;
     i = seq;
-    if (seq < n) { start = offs[seq]; L = offs[seq + 1] - start; nti = (L + BT - 1) / BT; }
+    if (seq < n) { start = win.start(seq); L = win.len(seq); nti = (L + BT - 1) / BT; }
   }
   __device__ void next() {
     if (++k == nti) { k = 0; load(i + 1); }
@@ -147,7 +160,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   }
   auto cursor = [&]() {
     TileCursor cur;
-    cur.offs = p.offs; cur.n = p.n_seq; cur.k = k0;
+    cur.win = p.win; cur.n = p.n_seq; cur.k = k0;
     cur.load(i0);
     return cur;
   };
@@ -319,7 +332,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float c = p.scale_log2;
     const float thr_add = kRescaleLog2 / c;
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l = 0.f, piece_max = -INFINITY;
     bool ok = true;
     TileCursor cur = cursor();
     // The loop runs the same named barriers in every thread whatever
@@ -359,6 +372,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
             }
           }
           const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+          piece_max = fmaxf(piece_max, mx);
           need = mx > m_used + thr_add;                     // always on a piece's first tile
           m_new = need ? mx : m_used;
           corr = need ? ex2((m_used - m_new) * c) : 1.f;    // 0 on a piece's first tile
@@ -441,12 +455,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
           if (head) {
             p.part_ml[(id * HEADS + x) * 2 + 0] = m_used;
             p.part_ml[(id * HEADS + x) * 2 + 1] = l;
+            // Prefill: the head's largest scaled logit (order-independent atomic max).
+            if (p.maxlogit && piece_max > -INFINITY) atomic_max_float(p.maxlogit + x, piece_max * p.scale);
           }
           tc_fence_before();
           mbar_arrive(bar(UFREE));
         }
         m_used = -INFINITY;
         l = 0.f;
+        piece_max = -INFINITY;
       }
       cur.next();
     }
@@ -462,7 +479,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
 // Work plan of the split kernel, built by one block of 256 threads:
 //   plan[0..n]        P_i = number of BT-token tiles of sequences 0..i-1
 //   plan[n+1+c]       the sequence holding tile floor(c P_n / G), c < G
-__device__ void build_plan(int n_seq, const int* __restrict__ offs, int G, int* __restrict__ plan) {
+__device__ void build_plan(int n_seq, Windows win, int G, int* __restrict__ plan) {
   __shared__ int wsum[8];
   __shared__ int carry;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -470,7 +487,7 @@ __device__ void build_plan(int n_seq, const int* __restrict__ offs, int G, int* 
   __syncthreads();
   for (int base = 0; base < n_seq; base += 256) {
     const int i = base + (int)threadIdx.x;
-    int x = i < n_seq ? (offs[i + 1] - offs[i] + BT - 1) / BT : 0;
+    int x = i < n_seq ? (win.len(i) + BT - 1) / BT : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -510,7 +527,7 @@ constexpr size_t ABS_SMEM = (size_t)(ABS_Q + ABS_SEQ) * LDK * 2;
 // Block (HEADS, 0, 0) builds the split kernel's work plan meanwhile.
 __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ W_UKV,
-                                                     __nv_bfloat16* __restrict__ q_abs, const int* __restrict__ offs,
+                                                     __nv_bfloat16* __restrict__ q_abs, Windows win,
                                                      int G, int* __restrict__ plan) {
   extern __shared__ __align__(16) uint8_t asm_[];
   __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(asm_);      // [128][LDK]: W_UK,h[latent][k]
@@ -520,7 +537,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(int n_seq, const __nv_bfloa
   constexpr size_t ldw = (size_t)HEADS * 256;
   griddep_launch_dependents();                 // the split kernel may be scheduled (it waits for this grid)
   if (h == HEADS) {                            // the extra column of blocks: one of them builds the plan
-    if (blockIdx.y == 0 && blockIdx.z == 0) build_plan(n_seq, offs, G, plan);
+    if (blockIdx.y == 0 && blockIdx.z == 0) build_plan(n_seq, win, G, plan);
     return;
   }
   for (int e = threadIdx.x; e < ABS_Q * 16; e += blockDim.x) {

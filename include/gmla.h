@@ -204,6 +204,29 @@ int mla_decode_absorbed(const gmla_geom* geom, gmla_dtype dtype, int n_seq,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mla_attn_fwd_absorbed — mla_attn_fwd's outputs (O and maxlogit[H]) computed
+ * on the latent cache instead of the materialised keys and values: every
+ * query is absorbed (q~_h = [q^C_h W_UK,h^T | q^S_h], 576 wide) and attends to
+ * the cache rows of its causal prefix, and the latent-space output is
+ * projected by W_UV,h.  This is the inference form of "Kimi Qkclip" (Fireworks
+ * blog), section 3, "Training vs. Inference in Multi-Head Latent Attention",
+ * applied to a prefill: K^C and V are never written to memory, at the price of
+ * (576 + 512) instead of (192 + 128) multiply-adds per query, key and head.
+ *   Q      [B][T][H][d_c + d_s]   W_UKV [kv_lora][H*(d_c+d_v)]
+ *   cache  [B][T][kv_lora + d_s] = [RMSNorm(c^KV) | k^S]  (mla_up_proj's `cache`)
+ *   g [B][T][H*d_v] or NULL;  O [B][T][H*d_v] (written)
+ *   maxlogit: device float[H], overwritten with max over b, t, s <= t of the
+ *     scaled logit, as mla_attn_fwd defines it.
+ *   workspace: at least mla_attn_fwd_absorbed_workspace() bytes.
+ * bf16 and Kimi K3's decode geometry only (H = 96, kv_lora = 512, d_c = 128,
+ * d_s = 64, d_v = 128), B * T <= 2^24; otherwise GMLA_EUNSUPPORTED.
+ */
+size_t mla_attn_fwd_absorbed_workspace(const gmla_geom* geom, int B, int T);
+int mla_attn_fwd_absorbed(const gmla_geom* geom, gmla_dtype dtype, int B, int T, const void* Q,
+                          const void* W_UKV, const void* cache, const void* g, void* O, float* maxlogit,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * mla_decode_absorbed_noalloc — mla_decode_absorbed for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is a deployment
  * variant.  Some callers cannot provide a workspace: a serving loop that must

@@ -100,6 +100,18 @@ def test_host_validation_without_gpu(lib):
     assert lib.mla_up_proj(G, 0, 2, 3, *([ok] * 10), None, None, ok, wsu, None) == -1
     assert lib.mla_gemm(0, 0, 4, 4, ok, ok, ok, None) == -1
     assert lib.mla_gemm(0, 4, 4, 4, ok, bad, ok, None) == -2
+    # absorbed prefill: K3 decode geometry and bf16 only; every pointer but g required; workspace checked
+    wsa = lib.mla_attn_fwd_absorbed_workspace(G, 1, 8)
+    assert wsa > 0 and lib.mla_attn_fwd_absorbed_workspace(ctypes.byref(_geom(m.TINY)), 1, 8) == 0
+    absorbed = lambda **kw: [kw.get(n, ok) for n in ("Q", "W", "cache", "g", "O", "ml")]
+    assert lib.mla_attn_fwd_absorbed(G, 0, 1, 0, *absorbed(), ok, wsa, None) == -1
+    assert lib.mla_attn_fwd_absorbed(G, 0, 1, 8, *absorbed(cache=None), ok, wsa, None) == -1
+    assert lib.mla_attn_fwd_absorbed(G, 0, 1, 8, *absorbed(ml=None), ok, wsa, None) == -1
+    assert lib.mla_attn_fwd_absorbed(G, 0, 1, 8, *absorbed(O=bad), ok, wsa, None) == -2
+    assert lib.mla_attn_fwd_absorbed(G, 1, 1, 8, *absorbed(), ok, wsa, None) == -3
+    assert lib.mla_attn_fwd_absorbed(ctypes.byref(_geom(m.TINY)), 0, 1, 8, *absorbed(), ok, wsa, None) == -3
+    assert lib.mla_attn_fwd_absorbed(G, 0, 1, 8, *absorbed(), ok, wsa - 1, None) == -6
+    assert lib.mla_attn_fwd_absorbed(G, 0, 1, 8, *absorbed(g=None), None, wsa, None) == -6
     # workspace queries reject bad sizes with 0
     assert lib.mla_decode_workspace(G, 0, 0, 100) == 0
     assert lib.mla_up_proj_workspace(None, 0, 1, 1) == 0

@@ -73,6 +73,9 @@ def _calls():
             geom=g, q=_t((NSEQ, g.H, g.d_qk)), W_UKV=W["W_UKV"], cache=_t((TOK, g.kv_lora + g.d_s)),
             seq_offsets=torch.tensor([0, 2, 9, 11], dtype=torch.int32), max_len=7, g=_t((NSEQ, g.H * g.d_v)),
             O=_t((NSEQ, g.H, g.d_v)))),
+        "mla_attn_fwd_absorbed": (gm.mla_attn_fwd_absorbed, dict(
+            geom=g, Q=attn["Q"], W_UKV=W["W_UKV"], cache=_t((B, T, g.kv_lora + g.d_s)), g=attn["g"],
+            O=_t((B, T, g.H * g.d_v)), maxlogit=_t(g.H, f32), workspace=_t(256, torch.uint8))),
         "mla_gemm": (gm.mla_gemm, dict(A=_t((7, 24)), B=_t((24, 16)), C=_t((7, 16)))),
     }
 
