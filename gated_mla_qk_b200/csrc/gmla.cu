@@ -296,7 +296,16 @@ static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfl
   if (M >= tc_gemm::PAIR_BM) {
     const long long tiles = tiles_n * ((M + tc_gemm::PAIR_BM - 1) / tc_gemm::PAIR_BM);
     const unsigned pairs = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms / 2));
-    tc_gemm::gemm_pair_kernel<<<2 * pairs, 192, tc_gemm::PAIR_SMEM_BYTES, st>>>(mA, mB, p);
+    // Output maps for the epilogue's tile stores: C, or K^C and V as [M][H * 128].
+    CUtensorMap mC0, mC1;
+    if (mode == 1) {
+      GMLA_TRY(make_map_2d(&mC0, KC, (uint64_t)H * 128, (uint64_t)M, 32));
+      GMLA_TRY(make_map_2d(&mC1, V, (uint64_t)H * 128, (uint64_t)M, 32));
+    } else {
+      GMLA_TRY(make_map_2d(&mC0, C, (uint64_t)N, (uint64_t)M, 32));
+      mC1 = mC0;
+    }
+    tc_gemm::gemm_pair_kernel<<<2 * pairs, 192, tc_gemm::PAIR_SMEM_BYTES, st>>>(mA, mB, mC0, mC1, p);
   } else {
     const long long tiles = tiles_n * ((M + tc_gemm::BM - 1) / tc_gemm::BM);
     const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms));

@@ -192,7 +192,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 // 16 KB of B from L2 instead of 16 + 32 KB, for the same tensor work.
 //   warp 0: TMA producer (both CTAs; the even CTA's full barrier counts both)
 //   warp 1: TMEM allocation (both CTAs), MMA issue (even CTA)
-//   warps 2-5: epilogue (both CTAs), as in gemm_kernel
+//   warps 2-5: epilogue (both CTAs): TMEM -> bf16 in swizzled shared memory
+//              -> TMA tile stores, the accumulator released after its last
+//              TMEM read, before the stores complete
 // Every wait is bounded; a pair has no early exit, so that both CTAs always
 // reach the cluster barriers and the paired TMEM allocation and release.
 // ===========================================================================
@@ -200,14 +202,17 @@ constexpr int PAIR_BM = 256, PAIR_NSTAGE = 6;              // pair tile rows; ri
 constexpr uint32_t PAIR_A_BYTES = 128 * BK * 2;             // this SM's 128 rows: 16 KB
 constexpr uint32_t PAIR_B_BYTES = 2 * BSUB;                 // this SM's 128 columns: 16 KB
 constexpr uint32_t PAIR_STAGE = PAIR_A_BYTES + PAIR_B_BYTES;  // 32 KB
-constexpr uint32_t PAIR_OFF_EPI = PAIR_NSTAGE * PAIR_STAGE;
-constexpr uint32_t PAIR_OFF_BAR = PAIR_OFF_EPI + 4 * EPI_WARP;
+constexpr uint32_t PAIR_EPI_BUF = 32 * 128;                  // [32 rows][64 cols] bf16, 128-byte swizzle: 4 KB
+constexpr uint32_t PAIR_OFF_EPI = PAIR_NSTAGE * PAIR_STAGE;  // 4 epilogue warps x 2 staging buffers
+constexpr uint32_t PAIR_OFF_BAR = PAIR_OFF_EPI + 8 * PAIR_EPI_BUF;
 constexpr uint32_t PAIR_SMEM_BYTES = PAIR_OFF_BAR + 256 + 1024;
+static_assert(PAIR_SMEM_BYTES + 64 <= 232448, "pair GEMM shared memory exceeds the per-block limit");
 enum PairBar { PFULL = 0, PEMPTY = PAIR_NSTAGE, PACCF = 2 * PAIR_NSTAGE, PACCE = PACCF + 2, PDRAIN = PACCE + 2,
                PNBAR = PDRAIN + 1 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1, Params p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -287,9 +292,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     __syncwarp();
   } else {
-    // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) .. + 31 = this SM's rows
+    // epilogue warps 2..5: TMEM lanes 32 * (warp % 4) .. + 31 = this SM's rows.
+    // Each 64-column chunk is rounded to bf16 into one of the warp's two
+    // swizzled staging buffers and written by one TMA tile store (elements
+    // past M or N are not written).  The accumulator is released as soon as
+    // its last chunk has been read from TMEM; the stores run on behind it.
     const int sub = warp & 3;
-    int j = 0;
+    const uint32_t stg0 = sbase + PAIR_OFF_EPI + (uint32_t)sub * 2u * PAIR_EPI_BUF;
+    if (lane == 0) { tma_prefetch_desc(&tmC0); tma_prefetch_desc(&tmC1); }
+    int j = 0, chunk = 0;
+    int last_buf = -1;                             // lane 0: staging buffer of the latest committed store
     for (int tile = pair_id; tile < n_tiles; tile += n_pairs, ++j) {
       const int acc = j & 1;
       const bool w = mbar_wait(bar(PACCF + acc), (uint32_t)(j >> 1) & 1u, abort);
@@ -297,49 +309,51 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc_fence_after();
       const int tn = tile % n_tiles_n, tm = tile / n_tiles_n;
       const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + 256u * (uint32_t)acc;
-      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem_raw + (sbase - sraw) + PAIR_OFF_EPI + sub * EPI_WARP);
       const int row0 = tm * PAIR_BM + 128 * (int)rank + sub * 32;
 #pragma unroll 1
-      for (int q = 0; q < BN / 64; ++q) {
+      for (int q = 0; q < BN / 64; ++q, ++chunk) {
         float v[64];
         tmem_ld32(taddr + 64u * q, *reinterpret_cast<float(*)[32]>(&v[0]));
         tmem_ld32(taddr + 64u * q + 32u, *reinterpret_cast<float(*)[32]>(&v[32]));
         tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&v[0]));
         tmem_wait_ld_dep(*reinterpret_cast<float(*)[32]>(&v[32]));
+        if (q == BN / 64 - 1) {
+          // Accumulator acc is free once both SMs' epilogues have read it (256 arrivals on the even CTA).
+          tc_fence_before();
+          if (rank == 0) mbar_arrive(bar(PACCE + acc));
+          else mbar_arrive_cluster(map_to_cta(bar(PACCE + acc), 0));
+        }
+        const int b = chunk & 1;
+        const uint32_t buf = stg0 + (uint32_t)b * PAIR_EPI_BUF;
+        // Every store but the latest has finished reading its buffer; the
+        // latest must have too if it read this one (chunks past N store nothing).
+        if (lane == 0) {
+          if (last_buf == b) bulk_wait_group_read<0>();
+          else bulk_wait_group_read<1>();
+        }
         __syncwarp();
-        uint4* srow = reinterpret_cast<uint4*>(stg + lane * EPI_LD);
+        const uint32_t srow = buf + (uint32_t)lane * 128u;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          srow[c] = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
-                               pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+          st_shared_v4(srow + ((uint32_t)(c ^ (lane & 7)) << 4), pack_bf16x2(v[8 * c], v[8 * c + 1]),
+                       pack_bf16x2(v[8 * c + 2], v[8 * c + 3]), pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
+                       pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+        fence_proxy_async_smem();
         __syncwarp();
-        const int col = tn * BN + 64 * q + 8 * (lane & 7);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = 4 * i + (lane >> 3);
-          const int row = row0 + r;
-          if (row >= p.M || col >= p.N) continue;
-          const uint4 val = reinterpret_cast<const uint4*>(stg + r * EPI_LD)[lane & 7];
-          __nv_bfloat16* dst;
-          if (p.mode == 1) {
-            const int h = col / 256, jj = col % 256;
-            dst = (jj < 128) ? p.KC + ((size_t)row * p.H + h) * 128 + jj : p.V + ((size_t)row * p.H + h) * 128 + (jj - 128);
-          } else {
-            dst = p.C + (size_t)row * p.N + col;
-          }
-          if (col + 8 <= p.N) {
-            *reinterpret_cast<uint4*>(dst) = val;
-          } else {
-            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&val);
-            for (int k = 0; k < 8 && col + k < p.N; ++k) dst[k] = e[k];
+        if (lane == 0) {
+          // mode 1: chunks 0-1 of head tn's tile are K^C_tn, chunks 2-3 are V_tn.
+          const CUtensorMap* m = (p.mode == 1 && q >= 2) ? &tmC1 : &tmC0;
+          const int x = p.mode == 1 ? tn * 128 + 64 * (q & 1) : tn * BN + 64 * q;
+          if (row0 < p.M && (p.mode == 1 || x < p.N)) {
+            tma_store_2d(m, buf, x, row0);
+            bulk_commit_group();
+            last_buf = b;
           }
         }
       }
-      // Accumulator acc is free once both SMs' epilogues have read it (256 arrivals on the even CTA).
-      tc_fence_before();
-      if (rank == 0) mbar_arrive(bar(PACCE + acc));
-      else mbar_arrive_cluster(map_to_cta(bar(PACCE + acc), 0));
     }
+    if (lane == 0) bulk_wait_group_all();          // every store has left shared memory and landed
+    __syncwarp();
   }
   tc_fence_before();
   cluster_sync();                      // both CTAs done with the accumulators and the ring
