@@ -14,6 +14,8 @@ pytestmark = pytest.mark.gpu
     (200, 576, 7168),      # ragged M, N = 2 tiles + 64 (the joint KV down-projection width)
     (1, 1536, 1536),       # a single row
     (300, 264, 520),       # ragged everything (N, K multiples of 8)
+    (257, 520, 64),        # one row past a 256-row pair tile; the last 64-column store box holds 8 columns
+    (512, 72, 128),        # N below one 256-column tile: a full box, an 8-column box, two boxes past N
     (1024, 2048, 512),
     (4096, 6144, 1536),    # 768 output tiles: every persistent CTA walks five or six, both TMEM accumulators cycle
 ])

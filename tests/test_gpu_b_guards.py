@@ -108,7 +108,7 @@ def test_decode_guards(lens, gate):
     O2.check("O (fixed scratch)")
 
 
-@pytest.mark.parametrize("M,N,K,dtype", [(300, 264, 520, "bf16"), (1, 1536, 1536, "bf16"), (129, 8, 8, "bf16"),
+@pytest.mark.parametrize("M,N,K,dtype", [(300, 264, 520, "bf16"), (512, 72, 128, "bf16"), (1, 1536, 1536, "bf16"), (129, 8, 8, "bf16"),
                                          (70, 45, 33, "f32")])
 def test_gemm_guards(M, N, K, dtype):
     import torch
