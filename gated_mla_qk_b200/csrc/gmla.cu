@@ -264,8 +264,11 @@ static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const vo
 // bf16 GEMM on the tensor cores when the shapes suit TMA (row strides of
 // whole 16-byte units), else the CUDA-core GEMM.  mode 1 writes the per-head
 // [K^C_h | V_h] split of an N = H * 256 product.
+// N2 > 0 (plain mode, from 256 rows on, N2 % 8 == 0): a second product
+// C2 = A B2 [M][N2] runs in the same pair launch (see gemm_bf16_two).
 static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfloat16* B, __nv_bfloat16* C,
-                     __nv_bfloat16* KC, __nv_bfloat16* V, int H, int d_c, int d_v, int mode, cudaStream_t st) {
+                     __nv_bfloat16* KC, __nv_bfloat16* V, int H, int d_c, int d_v, int mode, cudaStream_t st,
+                     int N2 = 0, const __nv_bfloat16* B2 = nullptr, __nv_bfloat16* C2 = nullptr) {
   const bool tc = (K % 8 == 0) && (N % 8 == 0) && (mode == 0 || (d_c == 128 && d_v == 128));
   if (!tc) {
     if (mode == 1) return simt::gemm<__nv_bfloat16>(M, N, K, A, B, simt::EpiSplitKV<__nv_bfloat16>{KC, V, H, d_c, d_v}, st);
@@ -282,21 +285,23 @@ static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfl
     return e;
   });
   if (ae != cudaSuccess) return cuda_status(ae);
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mB2;
   GMLA_TRY(make_map_2d(&mA, A, (uint64_t)K, (uint64_t)M, tc_gemm::BM));
   GMLA_TRY(make_map_2d(&mB, B, (uint64_t)N, (uint64_t)K, tc_gemm::BK));
+  mB2 = mB;
+  if (N2 > 0) GMLA_TRY(make_map_2d(&mB2, B2, (uint64_t)N2, (uint64_t)K, tc_gemm::BK));
   tc_gemm::Params p;
-  p.M = M; p.N = N; p.K = K; p.C = C; p.KC = KC; p.V = V; p.H = H; p.mode = mode;
+  p.M = M; p.N = N; p.K = K; p.C = C; p.KC = KC; p.V = V; p.H = H; p.mode = mode; p.N2 = N2;
   // Persistent: one CTA per SM (never more CTAs than output tiles); from 256
   // rows on, CTA pairs on 256 x 256 tiles.
   int dev = 0, sms = 0;
   GMLA_TRY(cuda_status(cudaGetDevice(&dev)));
   GMLA_TRY(cuda_status(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)));
-  const long long tiles_n = (N + tc_gemm::BN - 1) / tc_gemm::BN;
+  const long long tiles_n = (N + tc_gemm::BN - 1) / tc_gemm::BN + (N2 + tc_gemm::BN - 1) / tc_gemm::BN;
   if (M >= tc_gemm::PAIR_BM) {
     const long long tiles = tiles_n * ((M + tc_gemm::PAIR_BM - 1) / tc_gemm::PAIR_BM);
     const unsigned pairs = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms / 2));
-    // Output maps for the epilogue's tile stores: C, or K^C and V as [M][H * 128].
+    // Output maps for the epilogue's tile stores: C (and C2), or K^C and V as [M][H * 128].
     CUtensorMap mC0, mC1;
     if (mode == 1) {
       GMLA_TRY(make_map_2d(&mC0, KC, (uint64_t)H * 128, (uint64_t)M, 32));
@@ -304,15 +309,28 @@ static int gemm_bf16(int M, int N, int K, const __nv_bfloat16* A, const __nv_bfl
     } else {
       GMLA_TRY(make_map_2d(&mC0, C, (uint64_t)N, (uint64_t)M, 32));
       mC1 = mC0;
+      if (N2 > 0) GMLA_TRY(make_map_2d(&mC1, C2, (uint64_t)N2, (uint64_t)M, 32));
     }
-    tc_gemm::gemm_pair_kernel<<<2 * pairs, 192, tc_gemm::PAIR_SMEM_BYTES, st>>>(mA, mB, mC0, mC1, p);
+    tc_gemm::gemm_pair_kernel<<<2 * pairs, 192, tc_gemm::PAIR_SMEM_BYTES, st>>>(mA, mB, mB2, mC0, mC1, p);
   } else {
+    if (N2 > 0) return GMLA_EINVAL;              // the caller runs the two products separately here
     const long long tiles = tiles_n * ((M + tc_gemm::BM - 1) / tc_gemm::BM);
     const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms));
     tc_gemm::gemm_kernel<<<grid, 192, tc_gemm::SMEM_BYTES, st>>>(mA, mB, p);
   }
   note_launches(1);
   return check_launch();
+}
+
+// C1 = A B1 [M][N1] and C2 = A B2 [M][N2], both plain: one pair launch over
+// the column tiles of both products when it applies (A read once, one last
+// wave for both), else two launches.
+static int gemm_bf16_two(int M, int N1, int N2, int K, const __nv_bfloat16* A, const __nv_bfloat16* B1,
+                         __nv_bfloat16* C1, const __nv_bfloat16* B2, __nv_bfloat16* C2, cudaStream_t st) {
+  if (M >= tc_gemm::PAIR_BM && K % 8 == 0 && N1 % 8 == 0 && N2 % 8 == 0)
+    return gemm_bf16(M, N1, K, A, B1, C1, nullptr, nullptr, 0, 0, 0, 0, st, N2, B2, C2);
+  GMLA_TRY(gemm_bf16(M, N1, K, A, B1, C1, nullptr, nullptr, 0, 0, 0, 0, st));
+  return gemm_bf16(M, N2, K, A, B2, C2, nullptr, nullptr, 0, 0, 0, 0, st);
 }
 
 template <typename T>
@@ -333,9 +351,15 @@ int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, c
     else
       return simt::gemm<T>(Mm, N, K, A, B, simt::EpiPlain<T>{C, N}, st);
   };
-  GMLA_TRY(plain(M, g->q_lora, g->d_model, x, W_DQ, cQ));
-  // bf16 K3 widths: one warp per row (simt.cuh); otherwise one block per row.
+  // The two products of x: c^Q = x W_DQ and [c^KV k^S] = x W_DKV.
   constexpr bool bf = std::is_same<T, __nv_bfloat16>::value;
+  if constexpr (bf) {
+    GMLA_TRY(gemm_bf16_two(M, g->q_lora, g->kv_lora + g->d_s, g->d_model, x, W_DQ, cQ, W_DKV, ckv, st));
+  } else {
+    GMLA_TRY(plain(M, g->q_lora, g->d_model, x, W_DQ, cQ));
+    GMLA_TRY(plain(M, g->kv_lora + g->d_s, g->d_model, x, W_DKV, ckv));
+  }
+  // bf16 K3 widths: one warp per row (simt.cuh); otherwise one block per row.
   if constexpr (bf) {
     if (g->q_lora == 1536)
       simt::norm_rows_bf16_kernel<6><<<(M + 7) / 8, 256, 0, st>>>(cQ, M, w_q, g->rms_eps, cQh);
@@ -346,7 +370,6 @@ int up_proj_impl(const gmla_geom* g, int B, int Tn, const T* x, const T* W_DQ, c
   }
   note_launches(1);
   GMLA_TRY(plain(M, g->H * d_qk, g->q_lora, cQh, W_UQ, Q));
-  GMLA_TRY(plain(M, g->kv_lora + g->d_s, g->d_model, x, W_DKV, ckv));
   if constexpr (bf) {
     if (g->kv_lora == 512 && g->d_s == 64)
       simt::norm_kv_rows_bf16_kernel<2><<<(M + 7) / 8, 256, 0, st>>>(ckv, M, w_kv, g->rms_eps, ckvh, kS, cache);

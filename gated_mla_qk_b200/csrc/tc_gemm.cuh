@@ -42,6 +42,7 @@ struct Params {
   __nv_bfloat16* V;          // [M][H][128] (mode 1)
   int H;
   int mode;                  // 0: plain, 1: per-head split of [K^C_h | V_h] (N = H * 256)
+  int N2;                    // pair kernel, mode 0: a second product A B2 [M][N2] in the same launch (0: none)
 };
 
 __global__ void __launch_bounds__(192, 1)
@@ -212,7 +213,8 @@ enum PairBar { PFULL = 0, PEMPTY = PAIR_NSTAGE, PACCF = 2 * PAIR_NSTAGE, PACCE =
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1, Params p) {
+                 const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmC0,
+                 const __grid_constant__ CUtensorMap tmC1, Params p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -223,7 +225,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();                 // 0: issues the pair's MMAs
   const int n_pairs = (int)(gridDim.x / 2), pair_id = (int)(blockIdx.x / 2);
-  const int n_tiles_n = (p.N + BN - 1) / BN;
+  // Column tiles of the first product, then (N2 > 0) of the second, which
+  // shares A: one walk over both, so A is read once and the two products
+  // share their last wave.
+  const int n_tiles_n1 = (p.N + BN - 1) / BN;
+  const int n_tiles_n = n_tiles_n1 + (p.N2 + BN - 1) / BN;
   const int n_tiles = n_tiles_n * ((p.M + PAIR_BM - 1) / PAIR_BM);
   const int nk = (p.K + BK - 1) / BK;
 
@@ -241,10 +247,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
+      if (p.N2 > 0) tma_prefetch_desc(&tmB2);
       int it = 0;
       bool ok = true;
       for (int tile = pair_id; ok && tile < n_tiles; tile += n_pairs) {
         const int tn = tile % n_tiles_n, tm = tile / n_tiles_n;
+        const bool second = tn >= n_tiles_n1;
+        const CUtensorMap* mB = second ? &tmB2 : &tmB;
+        const int bcol = (second ? tn - n_tiles_n1 : tn) * BN + 128 * (int)rank;
         for (int k = 0; k < nk; ++k, ++it) {
           const uint32_t s = it % PAIR_NSTAGE, ph = (it / PAIR_NSTAGE) & 1;
           if (!mbar_wait(bar(PEMPTY + s), ph ^ 1u, abort)) { ok = false; break; }
@@ -253,7 +263,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if (rank == 0) mbar_arrive_expect_tx(bar(PFULL + s), 2 * PAIR_STAGE);
           tma_load_2d_pair(st, &tmA, full0, k * BK, tm * PAIR_BM + 128 * (int)rank);
           for (int c = 0; c < 2; ++c)
-            tma_load_2d_pair(st + PAIR_A_BYTES + c * BSUB, &tmB, full0, tn * BN + 128 * (int)rank + 64 * c, k * BK);
+            tma_load_2d_pair(st + PAIR_A_BYTES + c * BSUB, mB, full0, bcol + 64 * c, k * BK);
         }
       }
       // Never leave with copies in flight into this CTA's shared memory: a
@@ -341,10 +351,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          // mode 1: chunks 0-1 of head tn's tile are K^C_tn, chunks 2-3 are V_tn.
-          const CUtensorMap* m = (p.mode == 1 && q >= 2) ? &tmC1 : &tmC0;
-          const int x = p.mode == 1 ? tn * 128 + 64 * (q & 1) : tn * BN + 64 * q;
-          if (row0 < p.M && (p.mode == 1 || x < p.N)) {
+          // mode 1: chunks 0-1 of head tn's tile are K^C_tn, chunks 2-3 are
+          // V_tn (tmC0, tmC1).  mode 0: C (tmC0), or the second product's C2 (tmC1).
+          const bool second = tn >= n_tiles_n1;
+          const CUtensorMap* m = ((p.mode == 1 && q >= 2) || second) ? &tmC1 : &tmC0;
+          const int x = p.mode == 1 ? tn * 128 + 64 * (q & 1) : (second ? tn - n_tiles_n1 : tn) * BN + 64 * q;
+          if (row0 < p.M && (p.mode == 1 || x < (second ? p.N2 : p.N))) {
             tma_store_2d(m, buf, x, row0);
             bulk_commit_group();
             last_buf = b;
