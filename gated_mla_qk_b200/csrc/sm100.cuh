@@ -428,6 +428,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// The same for a 64-byte swizzle (layout = 4), K-major: rows of 64 B (32
+// bf16 along K), 16-byte chunk c of row r stored at chunk c ^ ((r >> 1) & 3);
+// SBO = 512 B between 8-row groups; the buffer 512-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_sw64_kmajor(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;                 // LBO unused for swizzled K-major operands
+  d |= (uint64_t)(512u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
+}
+
 // A descriptor moved by `bytes` (a multiple of 16).  The start-address field
 // holds address >> 4 in its low 14 bits; shared-memory addresses stay below
 // 256 KB, so the add never carries out of the field.  An issuing thread can

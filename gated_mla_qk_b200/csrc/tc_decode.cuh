@@ -24,12 +24,15 @@
 // score product (one softmax row per thread), the latent sits on M for the
 // value product, so U^T takes 4 x 96 TMEM columns beside the 96-column S.
 // q~ (108 KB) stays in shared memory for the whole sequence.  The tile's
-// latent streams through a ring of three 24 KB slots twice: once, as 128-wide
+// latent streams through a ring of four 24 KB slots twice: once, as 128-wide
 // latent pairs, for the score product, and once more (from L2, where the
 // first pass left it under an evict-last policy) for the value product after
 // the softmax, so no slot is held across the softmax and the ring stays short.  The 64 shared-key dims
-// have a slot of their own.  The score product of tile t+1 runs while the
-// softmax of tile t runs; S is released as soon as the softmax has loaded it.
+// are a fifth score-product item of the same ring (in the first half of a
+// slot).  P^T's last 32 tokens use a 64-byte swizzle (6 KB instead of 12),
+// which is what makes room for the fourth slot.  The score product of tile
+// t+1 runs while the softmax of tile t runs; S is released as soon as the
+// softmax has loaded it.
 // Softmax: base-2 exponentials against a lazily updated reference max per
 // head; U^T's column of a head is rescaled only when the head's max grows by
 // more than 2^8 (all four softmax warps take part, since a head's column
@@ -44,25 +47,30 @@ namespace tc_dec {
 using namespace sm100;
 
 constexpr int HEADS = 96, BT = 96, LAT = 512, WID = 576;
-constexpr int NPS = 3;                     // latent-pair ring slots
+constexpr int NPS = 4;                     // ring slots (latent pairs; the shared-key dims in half a slot)
 constexpr int G_CAP = 256;                 // most split CTAs (one per SM)
 constexpr uint32_t CSUB = BT * 128;        // [96 tokens x 64 dims] bf16, 12 KB
 constexpr uint32_t PAIR = 2 * CSUB;        // one 128-wide latent pair, 24 KB
 constexpr uint32_t QCH = HEADS * 128;      // [96 heads x 64 dims] bf16, 12 KB
 constexpr uint32_t OFF_Q = 0;              // q~: 9 chunks of 64 dims
-constexpr uint32_t OFF_P = OFF_Q + 9 * QCH;                 // P^T: two [96 heads x 64 tokens] sub-tiles
-constexpr uint32_t OFF_PAIR = OFF_P + 2 * QCH;
-constexpr uint32_t OFF_ROPE = OFF_PAIR + NPS * PAIR;
-constexpr uint32_t OFF_CORR = OFF_ROPE + CSUB;              // 96 rescale factors
+constexpr uint32_t OFF_P = OFF_Q + 9 * QCH;                 // P^T tokens 0-63: [96 heads x 64] 128-byte swizzle
+constexpr uint32_t OFF_P2 = OFF_P + QCH;                    // P^T tokens 64-95: [96 heads x 32] 64-byte swizzle
+constexpr uint32_t P2_BYTES = HEADS * 64;                   // 6 KB
+static_assert(BT == 96, "P^T is laid out as 64 + 32 tokens");
+constexpr uint32_t OFF_PAIR = OFF_P2 + P2_BYTES;
+constexpr uint32_t OFF_CORR = OFF_PAIR + NPS * PAIR;        // 96 rescale factors
 constexpr uint32_t OFF_BAR = OFF_CORR + 512;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr uint32_t TM_S = 0, TM_U = 128;   // TMEM columns: S (96), U^T 4 x 96
+static_assert(OFF_PAIR % 1024 == 0, "ring slots must be 1024-byte aligned (128-byte swizzle)");
+static_assert(OFF_P2 % 512 == 0, "the 64-byte swizzled P^T part must be 512-byte aligned");
+static_assert(SMEM_BYTES + 64 <= 232448, "decode shared memory exceeds the per-block limit");
 // The score product reads 128 rows of each q~ chunk: rows 96-127 fall on the
 // next chunk (or on P^T for the last one), and the S rows they give are never
 // read.
 
-enum Bar { QFULL = 0, QEMPTY, LFULL, LEMPTY = LFULL + NPS, RFULL = LEMPTY + NPS, REMPTY, SFULL, SFREE, PFULL,
-           PVDONE, UFREE, DRAIN, NBAR };
+enum Bar { QFULL = 0, QEMPTY, LFULL, LEMPTY = LFULL + NPS, SFULL = LEMPTY + NPS, SFREE, PFULL, PVDONE, UFREE,
+           DRAIN, NBAR };
 
 constexpr float kRescaleLog2 = 8.f;
 // Tiles brought into L2 ahead of their first ring load.  One is enough; at
@@ -166,8 +174,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
   };
 
   // Ring order (producer and MMA thread walk it alike): the score-product
-  // pairs of tile 0; then, per tile t, the score-product pairs of tile t+1
-  // followed by the value-product pairs of tile t.
+  // items of tile 0 (four latent pairs, then the shared-key dims); then, per
+  // tile t, the score-product items of tile t+1 followed by the value-product
+  // pairs of tile t.
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -184,7 +193,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
           pf.next();
         }
       };
-      int u = 0, seg = 0, rope_issued = 0;
+      int u = 0, seg = 0;
       bool ok = true;
       // The first pass over a tile keeps its lines in L2 for the second; the
       // second pass is their last use.
@@ -199,14 +208,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
         tma_load_2d_hint(dst + CSUB, &tmC, bar(LFULL + slot), 128 * pr + 64, row, pol);
         ++u;
       };
+      auto load_rope = [&](int row) {       // the 64 shared-key dims, first half of a slot
+        const uint32_t slot = (uint32_t)(u % NPS);
+        if (!mbar_wait(bar(LEMPTY + slot), ((uint32_t)(u / NPS) & 1u) ^ 1u, abort)) { ok = false; return; }
+        mbar_arrive_expect_tx(bar(LFULL + slot), CSUB);
+        tma_load_2d_hint(sbase + OFF_PAIR + slot * PAIR, &tmC, bar(LFULL + slot), LAT, row, pol_drop);   // read once
+        ++u;
+      };
       auto load_qk = [&](int t) {           // score-product items of tile t (cursor cq at t)
+        (void)t;
         const int row = cq.row();
         for (int pr = 0; pr < 4 && ok; ++pr) load_pair(row, pr, false);
-        if (!ok) return;
-        if (!mbar_wait(bar(REMPTY), ((uint32_t)t & 1u) ^ 1u, abort)) { ok = false; return; }
-        mbar_arrive_expect_tx(bar(RFULL), CSUB);
-        tma_load_2d(sbase + OFF_ROPE, &tmC, bar(RFULL), LAT, row);
-        ++rope_issued;
+        if (ok) load_rope(row);
       };
       prefetch_upto(kPrefetchAhead);
       mbar_arrive_expect_tx(bar(QFULL), 9 * QCH);
@@ -231,7 +244,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
       }
       // Never leave with copies in flight into this CTA's shared memory.
       mbar_wait_drain(bar(QFULL), (uint32_t)seg & 1u);
-      if (rope_issued > 0) mbar_wait_drain(bar(RFULL), (uint32_t)(rope_issued - 1) & 1u);
       for (int v = (u > NPS ? u - NPS : 0); v < u; ++v) mbar_wait_drain(bar(LFULL + v % NPS), (uint32_t)(v / NPS) & 1u);
     }
   } else if (warp == 5) {
@@ -249,8 +261,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
       // Base descriptors, built once: every MMA below steps one of them by a
       // compile-time byte offset (or picks a ring slot's).
       const uint64_t dQ = sdesc_sw128(sbase + OFF_Q, 16, 1024);
-      const uint64_t dRope = sdesc_sw128(sbase + OFF_ROPE, 16, 1024);
       const uint64_t dP = sdesc_sw128(sbase + OFF_P, 16, 1024);
+      const uint64_t dP2 = sdesc_sw64_kmajor(sbase + OFF_P2);
       const uint64_t dRingK = sdesc_sw128(sbase + OFF_PAIR, 16, 1024);     // slot 0, K-major (score B)
       const uint64_t dRingM = sdesc_sw128(sbase + OFF_PAIR, CSUB, 1024);   // slot 0, MN-major (value A)
       int slot_u = 0;                          // u % NPS and (u / NPS) & 1, kept incrementally
@@ -277,11 +289,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
                      (q | hf | kk) != 0);
           release_pair();
         }
-        if (!wait_ok(RFULL, (uint32_t)t & 1u)) return;
+        (void)t;
+        if (!next_pair()) return;              // the shared-key dims
+        {
+          const uint64_t sb = sdesc_add(dRingK, (uint32_t)slot_u * PAIR);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(d, sdesc_add(dQ, 8u * QCH + kk * 32u), sdesc_add(dRope, kk * 32u), idQK, true);
-        mma_commit(bar(REMPTY));
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(d, sdesc_add(dQ, 8u * QCH + kk * 32u), sdesc_add(sb, kk * 32u), idQK, true);
+        }
+        release_pair();
         mma_commit(bar(SFULL));
       };
       auto pv = [&](bool fresh) {
@@ -290,9 +306,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
           if (!next_pair()) return;
           const uint64_t sb = sdesc_add(dRingM, (uint32_t)slot_u * PAIR);
 #pragma unroll
-          for (int kk = 0; kk < BT / 16; ++kk)
+          for (int kk = 0; kk < BT / 16; ++kk)     // tokens 16 kk .. 16 kk + 15 of P^T
             mma_ss(tmem + TM_U + (uint32_t)b * HEADS, sdesc_add(sb, kk * 2048u),
-                   sdesc_add(dP, (uint32_t)(kk >> 2) * QCH + (uint32_t)(kk & 3) * 32u), idPV, !(fresh && kk == 0));
+                   kk < 4 ? sdesc_add(dP, (uint32_t)kk * 32u) : sdesc_add(dP2, (uint32_t)(kk - 4) * 32u), idPV,
+                   !(fresh && kk == 0));
           release_pair();
         }
         mma_commit(bar(PVDONE));
@@ -419,13 +436,16 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
         tmem_wait_st();
       }
       if (ok && head) {
-        // P^T row x: tokens 0-63 in the first sub-tile, 64-95 in the second.
+        // P^T row x: tokens 0-63 as a 128-byte row (128-byte swizzle), tokens
+        // 64-95 as a 64-byte row (64-byte swizzle).
+        const uint32_t prow = sbase + OFF_P + (uint32_t)x * 128u, prow2 = sbase + OFF_P2 + (uint32_t)x * 64u;
 #pragma unroll
-        for (int cc = 0; cc < BT / 8; ++cc) {
-          const uint32_t prow = sbase + OFF_P + (uint32_t)(cc >> 3) * QCH + (uint32_t)x * 128u;
-          st_shared_v4(prow + ((uint32_t)((cc & 7) ^ (x & 7)) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
-                       pk[4 * cc + 3]);
-        }
+        for (int cc = 0; cc < 8; ++cc)
+          st_shared_v4(prow + ((uint32_t)(cc ^ (x & 7)) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_shared_v4(prow2 + ((uint32_t)(cc ^ ((x >> 1) & 3)) << 4), pk[32 + 4 * cc], pk[33 + 4 * cc], pk[34 + 4 * cc],
+                       pk[35 + 4 * cc]);
       }
       if (ok) {
         fence_proxy_async_smem();
