@@ -462,6 +462,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
           tc_fence_after();
           const size_t id = (size_t)cta + (size_t)cur.i;
           float* dst = p.part_u + id * HEADS * LAT + x;
+          // The merge kernel reads the partials right after this kernel: keep
+          // them in L2 while the cache streams past under its own policies.
+          const uint64_t keep = l2_policy_evict_last();
 #pragma unroll 1
           for (int b = 0; b < 4; ++b)
 #pragma unroll 1
@@ -470,11 +473,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_consta
               tmem_ld32(tmem + lane_off + TM_U + (uint32_t)(b * HEADS + 32 * cc), u);
               tmem_wait_ld_dep(u);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) dst[(size_t)(32 * cc + e) * LAT + 128 * b] = u[e];
+              for (int e = 0; e < 32; ++e) st_global_hint(dst + (size_t)(32 * cc + e) * LAT + 128 * b, u[e], keep);
             }
           if (head) {
-            p.part_ml[(id * HEADS + x) * 2 + 0] = m_used;
-            p.part_ml[(id * HEADS + x) * 2 + 1] = l;
+            st_global_hint(p.part_ml + (id * HEADS + x) * 2 + 0, m_used, keep);
+            st_global_hint(p.part_ml + (id * HEADS + x) * 2 + 1, l, keep);
             // Prefill: the head's largest scaled logit (order-independent atomic max).
             if (p.maxlogit && piece_max > -INFINITY) atomic_max_float(p.maxlogit + x, piece_max * p.scale);
           }
