@@ -89,11 +89,12 @@ def test_tiny_fp32_layer_clip_and_recheck():
             assert ml_after[h] == ml_gpu[h]
 
 
-def test_up_proj_bf16_k3_geometry():
+@pytest.mark.parametrize("T", [100, 150])   # M = 200: two one-CTA launches for x's products; M = 300: one pair launch, ragged rows
+def test_up_proj_bf16_k3_geometry(T):
     geom = synth.K3
     rng = np.random.default_rng(21)
     W = {k: synth.round_storage(v, "bf16") for k, v in synth.layer_weights(geom, rng, with_gate_out=False).items()}
-    x = synth.round_storage(rng.standard_normal((2, 100, geom.d_model)).astype(np.float32), "bf16")
+    x = synth.round_storage(rng.standard_normal((2, T, geom.d_model)).astype(np.float32), "bf16")
     got = _up_proj_gpu(geom, "bf16", x, W)
     check_status()
     ref = oracle.up_proj(x, W["W_DQ"], W["w_q"], W["W_UQ"], W["W_DKV"], W["w_kv"], W["W_UKV"], geom, "bf16")
