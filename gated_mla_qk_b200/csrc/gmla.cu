@@ -254,9 +254,15 @@ static int attn_fwd_tc(const gmla_geom* g, int B, int T, const void* Q, const vo
   p.scale = 1.f / std::sqrt(192.f);
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(192.0));
   simt::fill_kernel<<<(H + 127) / 128, 128, 0, st>>>(maxlogit, H, -INFINITY);
+  // bf16 output: maps of the gate and of O for the epilogue's tile copies.
+  CUtensorMap mG = mQ, mO = mQ;
+  if (!out_f32) {
+    if (gate) GMLA_TRY(make_map_3d(&mG, gate, (uint64_t)H * 128, T, B));
+    GMLA_TRY(make_map_3d(&mO, O, (uint64_t)H * 128, T, B));
+  }
   const unsigned grid = (unsigned)p.n_qtiles * (unsigned)H * (unsigned)B;
-  if (out_f32) tc_attn::attn_fwd_kernel<true><<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, p);
-  else tc_attn::attn_fwd_kernel<false><<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, p);
+  if (out_f32) tc_attn::attn_fwd_kernel<true><<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, mG, mO, p);
+  else tc_attn::attn_fwd_kernel<false><<<grid, 192, tc_attn::SMEM_BYTES, st>>>(mQ, mKC, mKS, mV, mG, mO, p);
   note_launches(2);
   return check_launch();
 }

@@ -45,8 +45,11 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;     // + barriers + alignm
 
 // P_j and the P.V product of tile j hand off through PFULL + (j & 1) and
 // PVDONE + (j & 1): a softmax warp may run one tile ahead of the MMA issuer.
+// QEMPTY (gated bf16 form): every S product of the tile is done, so the Q
+// buffer is free for the gate tile (GFULL).  Without a gate the bf16 epilogue
+// stages O there after the last P.V product, which completes after every S.
 enum Bar { QFULL = 0, KVFULL = 1, KVEMPTY = KVFULL + NSTAGE, SFULL = KVEMPTY + NSTAGE, PFULL = SFULL + 2,
-           PVDONE = PFULL + 2, DRAIN = PVDONE + 2, NBAR = DRAIN + 1 };
+           PVDONE = PFULL + 2, QEMPTY = PVDONE + 2, GFULL, DRAIN, NBAR };
 
 constexpr float kRescaleLog2 = 8.f;   // rescale O when the row max grows by > 2^8
 
@@ -63,13 +66,18 @@ struct Params {
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
 
 // OUT_F32: the output is kept in fp32 (the training variant of "Gated MLA
-// et NoPE", "Un détail de précision numérique": no rounding of o to bf16).
-// The epilogue stores straight from registers, so no output tile occupies
-// shared memory in either variant.
+// et NoPE", "Un détail de précision numérique": no rounding of o to bf16);
+// that epilogue stores straight from registers.  The bf16 epilogue goes
+// through the Q buffer, free once the tile's last S product is done: the
+// producer loads the gate tile there (tmG) during the last steps, each
+// softmax thread turns its row of it into its row of o in place, and one
+// thread writes the tile with two TMA stores (tmO; rows past T are not
+// written).
 template <bool OUT_F32>
 __global__ void __launch_bounds__(192, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKC,
-                const __grid_constant__ CUtensorMap tmKS, const __grid_constant__ CUtensorMap tmV, Params p) {
+                const __grid_constant__ CUtensorMap tmKS, const __grid_constant__ CUtensorMap tmV,
+                const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmO, Params p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -103,6 +111,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     mbar_init(bar(PFULL + 1), 128);
     mbar_init(bar(PVDONE), 1);
     mbar_init(bar(PVDONE + 1), 1);
+    mbar_init(bar(QEMPTY), 1);
+    mbar_init(bar(GFULL), 1);
     mbar_init(bar(DRAIN), 1);
     fence_mbar_init();
   }
@@ -148,8 +158,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (j + 1 < n_kv) ok = load(true, j + 1);
         if (ok) ok = load(false, j);
       }
+      // bf16 epilogue: the gate tile into the Q buffer once Q is no longer read.
+      bool g_issued = false;
+      if constexpr (!OUT_F32) {
+        if (ok && p.g != nullptr && mbar_wait(bar(QEMPTY), 0, abort)) {
+          mbar_arrive_expect_tx(bar(GFULL), 2 * SUB);
+          tma_load_3d(sbase + OFF_Q, &tmG, bar(GFULL), kcol, qt * BM, b);
+          tma_load_3d(sbase + OFF_Q + SUB, &tmG, bar(GFULL), kcol + 64, qt * BM, b);
+          g_issued = true;
+        }
+      }
       // Never leave with copies in flight into this CTA's shared memory.
       mbar_wait_drain(bar(QFULL), 0);
+      if (g_issued) mbar_wait_drain(bar(GFULL), 0);
       for (uint32_t k = (u > NSTAGE ? u - NSTAGE : 0); k < u; ++k)
         mbar_wait_drain(bar(KVFULL + k % NSTAGE), (k / NSTAGE) & 1u);
     }
@@ -174,7 +195,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       };
       if (ok) {
         ok = mbar_wait(bar(KVFULL + 0), 0, abort);
-        if (ok) { tc_fence_after(); issue_S(0, 0); u = 1; }
+        if (ok) {
+          tc_fence_after();
+          issue_S(0, 0);
+          u = 1;
+          if (!OUT_F32 && p.g && n_kv == 1) mma_commit(bar(QEMPTY));   // the tile's last S product (gate staging)
+        }
       }
       for (int j = 0; ok && j < n_kv; ++j) {
         if (j + 1 < n_kv) {
@@ -183,6 +209,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
           issue_S((j + 1) & 1, slot);
           ++u;
+          if (!OUT_F32 && p.g && j + 2 == n_kv) mma_commit(bar(QEMPTY));   // the tile's last S product (gate staging)
         }
         if (!mbar_wait(bar(PFULL + (j & 1)), (uint32_t)(j >> 1) & 1u, abort)) { ok = false; break; }
         tc_fence_after();
@@ -291,23 +318,63 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tc_fence_before();
       mbar_arrive(bar(PFULL + buf));
     }
-    if (ok && wait_warp(PVDONE + ((n_kv - 1) & 1), (uint32_t)((n_kv - 1) >> 1) & 1u)) {
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool valid = t < p.T;
-      const size_t row_off = (((size_t)b * p.T + (valid ? t : 0)) * p.H + h) * 128;
+    const bool ep = ok && wait_warp(PVDONE + ((n_kv - 1) & 1), (uint32_t)((n_kv - 1) >> 1) & 1u);
+    const float inv_l = 1.f / l;
+    const bool valid = t < p.T;
+    if (ep) tc_fence_after();
+    if constexpr (OUT_F32) {
+      if (ep) {
+        const size_t row_off = (((size_t)b * p.T + (valid ? t : 0)) * p.H + h) * 128;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float o[32];
-        tmem_ld32(tO_row + 32u * k, o);
-        tmem_wait_ld_dep(o);
-        if (valid) {
-          const uint4* gp = reinterpret_cast<const uint4*>(p.g + row_off + 32 * k);
+        for (int k = 0; k < 4; ++k) {
+          float o[32];
+          tmem_ld32(tO_row + 32u * k, o);
+          tmem_wait_ld_dep(o);
+          if (valid) {
+            const uint4* gp = reinterpret_cast<const uint4*>(p.g + row_off + 32 * k);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              float gate[8];
+              if (p.g) {
+                uint4 gv = gp[v];
+                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = __bfloat1622float2(g2[e]);
+                  gate[2 * e] = sigmoidf_(f.x);
+                  gate[2 * e + 1] = sigmoidf_(f.y);
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gate[e] = 1.f;
+              }
+              float4* op = reinterpret_cast<float4*>(static_cast<float*>(p.O) + row_off + 32 * k) + 2 * v;
+              op[0] = make_float4(o[8 * v] * inv_l * gate[0], o[8 * v + 1] * inv_l * gate[1],
+                                  o[8 * v + 2] * inv_l * gate[2], o[8 * v + 3] * inv_l * gate[3]);
+              op[1] = make_float4(o[8 * v + 4] * inv_l * gate[4], o[8 * v + 5] * inv_l * gate[5],
+                                  o[8 * v + 6] * inv_l * gate[6], o[8 * v + 7] * inv_l * gate[7]);
+            }
+          }
+        }
+      }
+    } else {
+      // Row r of the staged tile: sub-tile k / 2 holds columns 64 (k / 2) ..,
+      // 16-byte chunk c of the row at chunk c ^ (r & 7) (128-byte swizzle).
+      const bool gated = p.g != nullptr;
+      const bool staged = ep && (!gated || wait_warp(GFULL, 0));
+      if (staged) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          float o[32];
+          tmem_ld32(tO_row + 32u * k, o);
+          tmem_wait_ld_dep(o);
+          const uint32_t rowb = sbase + OFF_Q + (uint32_t)(k >> 1) * SUB + (uint32_t)r * 128u;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
+            const uint32_t addr = rowb + ((uint32_t)((((k & 1) << 2) + v) ^ (r & 7)) << 4);
             float gate[8];
-            if (p.g) {
-              uint4 gv = gp[v];
+            if (gated) {
+              uint4 gv = ld_shared_v4(addr);
               const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -322,18 +389,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             float y[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) y[e] = o[8 * v + e] * inv_l * gate[e];
-            if constexpr (OUT_F32) {
-              float4* op = reinterpret_cast<float4*>(static_cast<float*>(p.O) + row_off + 32 * k) + 2 * v;
-              op[0] = make_float4(y[0], y[1], y[2], y[3]);
-              op[1] = make_float4(y[4], y[5], y[6], y[7]);
-            } else {
-              uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.O) + row_off + 32 * k);
-              op[v] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                                 pack_bf16x2(y[6], y[7]));
-            }
+            st_shared_v4(addr, pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                         pack_bf16x2(y[6], y[7]));
           }
         }
+        fence_proxy_async_smem();
       }
+      // Every softmax thread reaches this vote once, whatever happened above.
+      const bool all_staged = !bar_red_or(1, 128, !staged);
+      if (all_staged && r == 0) {
+        tma_store_3d(&tmO, sbase + OFF_Q, h * 128, qt * BM, b);
+        tma_store_3d(&tmO, sbase + OFF_Q + SUB, h * 128 + 64, qt * BM, b);
+        bulk_commit_group();
+        bulk_wait_group_read<0>();               // the tile has left shared memory (it lands before the grid completes)
+      }
+    }
+    if (ep) {
       if (p.lse && valid) p.lse[((size_t)b * p.T + t) * p.H + h] = fmaf(m_used, p.scale, __logf(l));
       float v = valid ? true_max * p.scale : -INFINITY;
 #pragma unroll
