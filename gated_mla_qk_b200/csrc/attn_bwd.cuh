@@ -57,6 +57,45 @@ __global__ void __launch_bounds__(256) row_kernel(int rows, int H, int d_v, cons
   if (lane == 0) D[row] = acc;
 }
 
+// The same row pass for d_v = 128 with a bf16 gate and bf16 dO~ (the tcgen05
+// backward's form): one warp per row, lane l takes columns 4l .. 4l+3 through
+// 16-byte fp32 and 8-byte bf16 accesses (4-byte accesses left the pass
+// latency-bound).  D sums each lane's four products first, then across lanes.
+__global__ void __launch_bounds__(256) row128_kernel(int rows, const float* __restrict__ O, const float* __restrict__ dO,
+                                                     const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ dOt,
+                                                     float* __restrict__ D, float* __restrict__ dg) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;                       // row = (b*T + t)*H + h
+  const size_t base = (size_t)row * 128 + 4 * lane;
+  const float4 d = *reinterpret_cast<const float4*>(dO + base);
+  const float4 o = *reinterpret_cast<const float4*>(O + base);
+  float acc = fmaf(d.w, o.w, fmaf(d.z, o.z, fmaf(d.y, o.y, d.x * o.x)));
+  float t[4] = {d.x, d.y, d.z, d.w};
+  if (g) {
+    const uint2 gv = *reinterpret_cast<const uint2*>(g + base);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+    const float2 ga = __bfloat1622float2(g2[0]), gb = __bfloat1622float2(g2[1]);
+    const float sg[4] = {1.f / (1.f + __expf(-ga.x)), 1.f / (1.f + __expf(-ga.y)), 1.f / (1.f + __expf(-gb.x)),
+                         1.f / (1.f + __expf(-gb.y))};
+    const float dv[4] = {d.x, d.y, d.z, d.w}, ov[4] = {o.x, o.y, o.z, o.w};
+    float q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      t[e] = dv[e] * sg[e];
+      q[e] = dv[e] * ov[e] * (1.f - sg[e]);
+    }
+    *reinterpret_cast<float4*>(dg + base) = make_float4(q[0], q[1], q[2], q[3]);
+  }
+  __nv_bfloat162 p0 = __floats2bfloat162_rn(t[0], t[1]), p1 = __floats2bfloat162_rn(t[2], t[3]);
+  uint2 out;
+  out.x = *reinterpret_cast<uint32_t*>(&p0);
+  out.y = *reinterpret_cast<uint32_t*>(&p1);
+  *reinterpret_cast<uint2*>(dOt + base) = out;
+#pragma unroll
+  for (int k = 16; k > 0; k >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, k);
+  if (lane == 0) D[row] = acc;
+}
+
 struct Dims {
   int B, T, H, d_c, d_s, d_v;
   float scale;

@@ -599,7 +599,7 @@ static int attn_bwd_tc(const bwd::Dims& d, const __nv_bfloat16* Q, const __nv_bf
   GMLA_TRY(make_map_3d(&mV64, V, (uint64_t)H * 128, T, B, 64));
   GMLA_TRY(cuda_status(cudaMemsetAsync(dkS, 0, (size_t)B * T * 64 * sizeof(float), st)));
   const int rows = B * T * H;
-  bwd::row_kernel<bf, bf><<<(rows + 7) / 8, 256, 0, st>>>(rows, H, 128, O, dO, gate, dOt, D, dg);
+  bwd::row128_kernel<<<(rows + 7) / 8, 256, 0, st>>>(rows, O, dO, static_cast<const bf*>(gate), dOt, D, dg);
   tc_bwd::Params p;
   p.B = B; p.T = T; p.H = H; p.lse = lse; p.D = D; p.dQ = dQ; p.dKC = dKC; p.dkS = dkS; p.dV = dV;
   p.scale = d.scale;
